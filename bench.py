@@ -1,0 +1,453 @@
+"""Benchmark of the SpecOPD branch-scoring hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  specopd_tree_build  (parent map, semantic positions, score rows)
+  specopd_tree_attn   (branch RoPE + tensor-core tree attention, one layer)
+  specopd_e2e_tv      (overlaps, prefix products, loss, d loss / d draft logits)
+on the 8B-shaped workload (T=4096, B=64 anchors over the response half, W=8,
+32 q / 8 kv heads, head_dim 128, bf16; vocab 151,936, N = 512 positions).
+The trunk K cache is rotated once before timing (it belongs to the trunk
+prefill, which runs once per trunk).
+
+Metric: scored branch rows per second, R = B(W-1) rows per step and per GPU.
+Multi-GPU (torchrun): every rank scores its own batch of branches (weak
+scaling); the only exchange is the distributed normalisation of the loss
+(one all-reduce of the prefix-product sum; the gradient already uses the
+global position count), as the method prescribes for ranks with different
+numbers of scored positions.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has: no implementation was released) on a bounded sample of the same
+workload, on this machine's host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "8b"
+METRIC = "scored branch rows/s (tree-attn + E2E-TV); % of bf16 TC peak and HBM roofline"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "src": "fallback"}
+
+
+def attention_flops(cfg, anchors):
+    """Algorithmic FLOPs: sum over rows and q heads of 4*D*(a_b + 1 + i)
+    (QK^T and PV over the visible keys only)."""
+    W = cfg.W
+    keys = 0
+    for a in anchors:
+        keys += sum(int(a) + 1 + i for i in range(1, W))
+    return 4.0 * cfg.D * cfg.Hq * keys
+
+
+def _clock_sampler(path):
+    cmd = ["nvidia-smi", "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"
+           "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+           "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+           "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "100"]
+    try:
+        f = open(path, "w")
+        return subprocess.Popen(cmd, stdout=f, stderr=subprocess.DEVNULL), f
+    except Exception:
+        return None, None
+
+
+def _clock_summary(path, dev_index):
+    sm, smax, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    try:
+        for line in open(path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9 or p[0] != str(dev_index):
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax = float(p[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+    except FileNotFoundError:
+        pass
+    return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ device problem
+
+class Problem:
+    """Device-resident inputs and outputs of one step (the 8B-shaped workload)."""
+
+    def __init__(self, torch, api, dev, seed_offset=0):
+        self.torch, self.api, self.dev = torch, api, dev
+        acfg = synth.attn_config(WORKLOAD)
+        tcfg = synth.tv_config(WORKLOAD)
+        self.acfg, self.tcfg = acfg, tcfg
+        inp = synth.attention_inputs(acfg)
+        self.inp = inp
+        bf = torch.bfloat16
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev).to(bf)  # noqa
+        self.cu_host = [int(c) for c in inp.cu_trunk]
+        self.cu_dev = torch.tensor(inp.cu_trunk, device=dev)
+        self.anchors = torch.tensor(inp.anchors, device=dev)
+        self.q_br, self.k_br, self.v_br = t(inp.q_br), t(inp.k_br), t(inp.v_br)
+        self.k_tr, self.v_tr = t(inp.k_tr), t(inp.v_tr)
+        S, B, W = acfg.S, acfg.B, acfg.W
+        self.R = S * B * (W - 1)
+        self.N = S * B * W
+        self.T_tot = inp.T_tot
+        i32 = torch.int32
+        self.parent = torch.empty(self.T_tot + self.R, dtype=i32, device=dev)
+        self.sem_pos = torch.empty(self.T_tot + self.R, dtype=i32, device=dev)
+        self.score_row = torch.empty(self.N, dtype=i32, device=dev)
+        api.specopd_tree_build(self.cu_host, self.anchors, B, W, self.parent, self.sem_pos,
+                               self.score_row)
+        # trunk K cache, rotated once (trunk prefill)
+        api.specopd_rope_apply(self.k_tr, self.sem_pos[: self.T_tot].contiguous(), acfg.rope_base)
+        self.desc = api.attn_desc(S, B, W, acfg.Hq, acfg.Hkv, acfg.D, "bf16", acfg.rope_base)
+        ws = api.specopd_tree_attn_workspace_size(self.desc, self.cu_host)
+        self.attn_ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.out = torch.empty_like(self.q_br)
+        # logits: target rows in packed node order [T_tot + R, V], read through
+        # the score-row map; draft logits [N, V].  Rows are generated on the
+        # device with the per-row recipe's distribution (seeded torch RNG), the
+        # oracle-checked rows come from synth on the host (tests).
+        V = tcfg.V
+        self.V = V
+        g = torch.Generator(device=dev)
+        g.manual_seed(1234 + seed_offset)
+        rows_t = self.T_tot + self.R
+        self.rows_t = rows_t
+        self.z_t = torch.zeros((rows_t, V), dtype=bf, device=dev)
+        zt = torch.randn((self.N, V), generator=g, device=dev) * tcfg.sigma_t
+        k = torch.randint(1, 4, (self.N,), generator=g, device=dev)
+        ids = torch.randint(0, V, (self.N, 3), generator=g, device=dev)
+        bump = (torch.arange(3, device=dev)[None, :] < k[:, None]).float() * tcfg.bump
+        zt.scatter_add_(1, ids, bump)
+        zd = zt + torch.randn((self.N, V), generator=g, device=dev) * tcfg.sigma_d
+        torch.cuda.synchronize()
+        sr = self.score_row.long()
+        self.z_t[sr] = zt.to(bf)
+        self.z_d = zd.to(bf)
+        del zt, zd
+        self.tdesc = api.tv_desc(S * B, W, V, rows_t, "bf16", "f32", True,
+                                 norm_count=self.N)
+        self.tv_ws = torch.empty(api.specopd_e2e_tv_workspace_size(self.tdesc), dtype=torch.uint8,
+                                 device=dev)
+        f32 = torch.float32
+        self.a = torch.empty(self.N, dtype=f32, device=dev)
+        self.prefix = torch.empty(self.N, dtype=f32, device=dev)
+        self.loss = torch.empty(1, dtype=f32, device=dev)
+        self.numer = torch.empty(1, dtype=torch.float64, device=dev)
+        self.grad = torch.empty((self.N, V), dtype=f32, device=dev)
+        self.flops = attention_flops(acfg, inp.anchors)
+        self.tv_bytes = float(self.N) * V * (2 + 2 + 4)
+
+    def step(self, ev=None):
+        api, acfg = self.api, self.acfg
+        api.specopd_tree_build(self.cu_host, self.anchors, acfg.B, acfg.W, self.parent,
+                               self.sem_pos, self.score_row)
+        if ev is not None:
+            ev[0].record()
+        api.specopd_tree_attn(self.desc, self.q_br, self.k_br, self.v_br, self.k_tr, self.v_tr,
+                              self.cu_dev, self.cu_host, self.anchors, self.sem_pos, out=self.out,
+                              workspace=self.attn_ws)
+        if ev is not None:
+            ev[1].record()
+        api.specopd_e2e_tv(self.tdesc, self.z_t, self.score_row, self.z_d, a=self.a,
+                           prefix=self.prefix, loss=self.loss, numer=self.numer, grad=self.grad,
+                           workspace=self.tv_ws)
+        if ev is not None:
+            ev[2].record()
+
+
+KERNELS_PER_STEP = 5  # tree_build, rope(q), rope(k), tree_attn, e2e_tv
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from tree_attention_specopd_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    api.load()
+    pb = Problem(torch, api, dev, seed_offset=rank)
+    if world > 1:
+        # Eq. 18: the gradient and loss divide by the GLOBAL position count.
+        pb.tdesc = api.tv_desc(pb.acfg.S * pb.acfg.B, pb.acfg.W, pb.V, pb.rows_t, "bf16", "f32",
+                               True, norm_count=pb.N * world)
+    numer_all = torch.zeros(1, dtype=torch.float64, device=dev)
+
+    def full_step(ev=None):
+        pb.step(ev)
+        if world > 1:
+            numer_all.copy_(pb.numer)
+            dist.all_reduce(numer_all)
+
+    for _ in range(args.warmup):
+        full_step()
+    torch.cuda.synchronize()
+    st = api.specopd_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x} after warm-up")
+
+    clk_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+    os.makedirs(os.path.dirname(clk_path), exist_ok=True)
+    sampler, fh = _clock_sampler(clk_path) if rank == 0 else (None, None)
+    time.sleep(0.3 if sampler else 0)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for k in range(args.steps):
+        full_step(evs[k])
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    attn_ms = sum(ev[0].elapsed_time(ev[1]) for ev in evs) / args.steps
+    tv_ms = sum(ev[1].elapsed_time(ev[2]) for ev in evs) / args.steps
+    if sampler:
+        sampler.terminate()
+        sampler.wait()
+        fh.close()
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    loss = float(pb.loss.item())
+    st = api.specopd_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x} after the timed steps")
+
+    # ---- end-to-end through the public API with host buffers
+    e2e = e2e_measure(torch, api, pb, args, dev, world)
+
+    if rank == 0:
+        peaks = _peaks()
+        ms_step = ms_max / args.steps
+        value = pb.R * world / (ms_step / 1e3)
+        tv_gbs = pb.tv_bytes / (tv_ms / 1e3) / 1e9
+        attn_tflops = pb.flops / (attn_ms / 1e3) / 1e12
+        clocks = _clock_summary(clk_path, local)
+        traffic = _ncu_traffic()
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "rows/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "8B-shaped single layer: T=4096, B=64 anchors, W=8, 32q/8kv "
+                                   "heads, head_dim 128, vocab 151936, N=512 positions",
+                       "rows_per_step_per_gpu": pb.R, "positions_per_step_per_gpu": pb.N,
+                       "parallelism": f"dp{world} (branch batches per rank)",
+                       "l2": "inputs larger than L2 (0.31 GB of logits read per step vs 126 MB)"},
+            "supervised_tokens_per_s": pb.N * world / (ms_step / 1e3),
+            "roofline": {"bound": "hbm", "kernel": "e2e_tv", "achieved": tv_gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": tv_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                         "algorithmic_bytes_per_launch": pb.tv_bytes, "launch_ms": tv_ms,
+                         "peak_src": peaks["src"]},
+            "attention_roofline": {"bound": "tensor", "kernel": "tree_attn", "achieved": attn_tflops,
+                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                   "frac": attn_tflops / peaks["bf16_tflops"],
+                                   "algorithmic_flops_per_launch": pb.flops, "launch_ms": attn_ms,
+                                   "peak_src": peaks["src"]},
+            "loss": loss,
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _ncu_traffic():
+    """DRAM bytes per e2e_tv launch from a committed ncu summary, if present."""
+    path = os.path.join(ROOT, "profiles", "e2e_tv_8b_traffic.json")
+    try:
+        return json.load(open(path))["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+def e2e_measure(torch, api, pb, args, dev, world):
+    """Same metric through the public API, host buffers: per step the branch
+    q/k/v, anchors and both logit batches are copied from pinned host memory,
+    and the loss is read back."""
+    import torch.distributed as dist
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    h = {"q": pin(pb.q_br), "k": pin(pb.k_br), "v": pin(pb.v_br), "anc": pin(pb.anchors),
+         "zt": pin(pb.z_t[pb.score_row.long()]), "zd": pin(pb.z_d)}
+    zt_rows = torch.empty_like(pb.z_d)
+    sr_long = pb.score_row.long()
+    loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = loss_h.numel() * 4
+
+    def one():
+        pb.q_br.copy_(h["q"], non_blocking=True)
+        pb.k_br.copy_(h["k"], non_blocking=True)
+        pb.v_br.copy_(h["v"], non_blocking=True)
+        pb.anchors.copy_(h["anc"], non_blocking=True)
+        zt_rows.copy_(h["zt"], non_blocking=True)
+        pb.z_d.copy_(h["zd"], non_blocking=True)
+        pb.z_t.index_copy_(0, sr_long, zt_rows)
+        pb.step()
+        loss_h.copy_(pb.loss, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    steps = max(2, min(args.steps, 10))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": pb.R * world / (ms / 1e3), "unit": "rows/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def cpu_baseline(seconds=15.0, nbranch=None):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload:
+    whole branches (their W-1 attention rows and W TV positions), timed on
+    the host cores; reported in the bench's unit (scored rows/s)."""
+    from oracle import attention as oatt
+    from oracle import tv as otv
+    acfg = synth.attn_config(WORKLOAD)
+    tcfg = synth.tv_config(WORKLOAD)
+    inp = synth.attention_inputs(acfg)
+    rows = 0
+    t0 = time.perf_counter()
+    b = 0
+    while True:
+        oatt.branch_attention_unrolled(inp.q_br, inp.k_br, inp.v_br, inp.k_tr, inp.v_tr,
+                                       inp.cu_trunk, inp.anchors, acfg.B, acfg.W,
+                                       acfg.rope_base, branches=[b])
+        zt, zd = synth.logits(tcfg, positions=range(b * acfg.W, (b + 1) * acfg.W))
+        otv.e2e_tv(zt, None, zd, 1, acfg.W, norm_count=tcfg.nbranch * acfg.W)
+        rows += acfg.W - 1
+        b += 1
+        el = time.perf_counter() - t0
+        if (nbranch is not None and b >= nbranch) or (nbranch is None and el >= seconds) \
+                or b >= acfg.B:
+            break
+    el = time.perf_counter() - t0
+    try:
+        import threadpoolctl
+        threads = max(int(x.get("num_threads", 1)) for x in threadpoolctl.threadpool_info()) \
+            if threadpoolctl.threadpool_info() else 1
+    except Exception:
+        threads = os.cpu_count()
+    return {"value": rows / el, "unit": "rows/s", "cores": threads, "kind": "oracle",
+            "sample": f"{b} of {acfg.B} branches of the 8B-shaped workload "
+                      f"({rows} rows, {b * acfg.W} TV positions) in {el:.1f} s; "
+                      f"host has {os.cpu_count()} cores"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per = []
+    for _ in range(args.warmup):
+        cpu_baseline(nbranch=1)
+    t0 = time.perf_counter()
+    rows = 0
+    for _ in range(args.steps):
+        r = cpu_baseline(nbranch=1)
+        rows += 7
+        per.append(r)
+    el = time.perf_counter() - t0
+    value = rows / el
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "8B-shaped single layer (one branch of it per step)"},
+            "cpu_baseline": {"value": value, "unit": "rows/s", "kind": "oracle",
+                             "cores": per[-1]["cores"] if per else os.cpu_count(),
+                             "sample": "1 branch (7 attention rows, 8 TV positions) per step"},
+            "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

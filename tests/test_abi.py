@@ -1,0 +1,61 @@
+"""The C-ABI library loads and exports every symbol include/specopd.h declares.
+
+CPU only: no compute call needs a GPU here; only host-side entry points
+(status strings, workspace sizes, argument validation that fails before any
+device work) are called.
+"""
+
+import ctypes
+
+import pytest
+
+from tree_attention_specopd_b200 import api, build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = api.header_functions()
+    assert len(names) == 9
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    assert lib.specopd_status_string(0) == b"SPECOPD_OK"
+    assert lib.specopd_status_string(3) == b"SPECOPD_ERR_WORKSPACE"
+    assert lib.specopd_status_string(99) == b"SPECOPD_ERR_UNKNOWN"
+    assert lib.specopd_version() == 10000
+
+
+def test_workspace_sizes_are_host_only(lib):
+    d = api.attn_desc(1, 64, 8, 32, 8, 128, "bf16")
+    n = api.specopd_tree_attn_workspace_size(d, [0, 4096])
+    assert n >= 448 * (32 + 8) * 128 * 2
+    t = api.tv_desc(64, 8, 151936, 4544, "bf16")
+    assert api.specopd_e2e_tv_workspace_size(t) >= 512 * 16
+    # invalid descriptors report 0
+    bad = api.attn_desc(1, 64, 8, 30, 8, 128, "bf16")  # Hq % Hkv != 0
+    assert api.specopd_tree_attn_workspace_size(bad, [0, 4096]) == 0
+    assert api.specopd_tree_attn_workspace_size(d, [1, 4096]) == 0  # cu[0] != 0
+    assert api.specopd_e2e_tv_workspace_size(api.tv_desc(0, 8, 100, 10, "f32")) == 0
+    # vocabularies too large for the cluster-resident rows are unsupported
+    assert api.specopd_e2e_tv_workspace_size(api.tv_desc(1, 1, 10_000_000, 1, "f32")) == 0
+
+
+def test_invalid_arguments_rejected_before_device(lib):
+    cu = (ctypes.c_int32 * 2)(0, 10)
+    # S = 0
+    assert lib.specopd_tree_build(0, cu, None, 1, 1, None, None, None, None) == 1
+    # non-increasing cu_trunk
+    bad = (ctypes.c_int32 * 2)(0, 0)
+    assert lib.specopd_tree_build(1, bad, ctypes.c_void_p(16), 1, 2, ctypes.c_void_p(16),
+                                  None, None, None) == 1
+    # rope with odd D
+    d = api.RopeDesc(7, 0, 10000.0)
+    assert lib.specopd_rope_apply(ctypes.byref(d), None, None, 4, 1, None) == 1

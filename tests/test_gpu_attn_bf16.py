@@ -1,0 +1,173 @@
+"""GPU parity of the bf16 tensor-core tree attention (tcgen05/TMEM/TMA kernel)
+against the fp64 unrolled oracle, through the C ABI.
+
+Tolerance: the target states 2e-2 absolute for bf16 attention outputs at
+unit-scale activations.  Because softmax averages thousands of unit-scale
+values, outputs are small (~0.03), so each test also bounds the normwise
+relative error max|err| / max|ref| by 1e-2: the inputs are bf16-exact, and
+the kernel rounds rotated q/k (2^-9 relative), P (2^-9) and the output
+(2^-9), which puts the expected error near 2e-3 of the output scale.
+Branch-dominant and masked-perturbation cases make the branch keys and the
+mask carry the result, where the average alone would hide a mistake.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import attention as oatt
+from tests._util import dev_tensor, rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+
+ATOL = 2e-2
+RTOL = 1e-2
+
+
+def _run(lib, inp, k_br=None, k_tr=None, v_tr=None, lse=False):
+    cfg = inp.cfg
+    dt = cfg.dtype
+    cu = [int(c) for c in inp.cu_trunk]
+    anchors = torch.tensor(inp.anchors, device="cuda")
+    _, sem_pos, _ = lib.specopd_tree_build(cu, anchors, cfg.B, cfg.W)
+    ktr = dev_tensor(inp.k_tr if k_tr is None else k_tr, dt)
+    lib.specopd_rope_apply(ktr, sem_pos[: inp.T_tot].contiguous(), cfg.rope_base)
+    desc = lib.attn_desc(cfg.S, cfg.B, cfg.W, cfg.Hq, cfg.Hkv, cfg.D, dt, cfg.rope_base)
+    lse_t = torch.empty((inp.R, cfg.Hq), dtype=torch.float32, device="cuda") if lse else None
+    out = lib.specopd_tree_attn(desc, dev_tensor(inp.q_br, dt),
+                                dev_tensor(inp.k_br if k_br is None else k_br, dt),
+                                dev_tensor(inp.v_br, dt), ktr,
+                                dev_tensor(inp.v_tr if v_tr is None else v_tr, dt),
+                                torch.tensor(inp.cu_trunk, device="cuda"), cu, anchors, sem_pos,
+                                lse=lse_t)
+    torch.cuda.synchronize()
+    return out, lse_t
+
+
+def _ref(inp, branches=None, k_br=None):
+    cfg = inp.cfg
+    return oatt.branch_attention_unrolled(inp.q_br, inp.k_br if k_br is None else k_br, inp.v_br,
+                                          inp.k_tr, inp.v_tr, inp.cu_trunk, inp.anchors, cfg.B,
+                                          cfg.W, cfg.rope_base, branches=branches)
+
+
+def _check(out, ref_by_branch, W, atol=ATOL, rtol=RTOL):
+    got = to_np(out)
+    for bid, ref in ref_by_branch.items():
+        g = got[bid * (W - 1): (bid + 1) * (W - 1)]
+        assert np.all(np.isfinite(g)), bid
+        assert np.max(np.abs(g - ref)) < atol, bid
+    allg = np.concatenate([got[b * (W - 1): (b + 1) * (W - 1)] for b in ref_by_branch])
+    allr = np.concatenate(list(ref_by_branch.values()))
+    assert rel_err(allg, allr) < rtol
+
+
+CASES = [
+    # S, T, B, W, Hq, Hkv, D
+    (2, (300, 520), 6, 5, 8, 2, 128),     # packed, G = 4, ragged tiles
+    (1, (700,), 9, 4, 10, 2, 128),        # G = 5 -> 25 rows x 5 heads = 125 MMA rows
+    (1, (260,), 20, 16, 4, 4, 128),       # G = 1: 128 rows/tile, two branch-key tiles
+    (1, (1000,), 5, 2, 16, 2, 64),        # D = 64, W = 2, G = 8
+    (3, (130, 2, 2000), 2, 3, 32, 8, 128),  # trunk of length 2, 8B head layout
+]
+
+
+@pytest.mark.parametrize("S,T,B,W,Hq,Hkv,D", CASES)
+def test_small_shapes(lib, S, T, B, W, Hq, Hkv, D):
+    cfg = synth.custom_attn_config(S, T, B, W, Hq, Hkv, D, "bf16", seed=S * 7 + W)
+    inp = synth.attention_inputs(cfg)
+    out, _ = _run(lib, inp)
+    _check(out, _ref(inp), W)
+    assert lib.specopd_get_device_status() == 0
+
+
+def test_edge_anchors_bf16(lib):
+    # a = 0, a = T-1, duplicates, unsorted anchors.
+    cfg = synth.custom_attn_config(2, (200, 333), 5, 4, 8, 2, 128, "bf16", seed=3)
+    anchors = [199, 0, 0, 57, 199, 332, 0, 100, 100, 17]
+    inp = synth.attention_inputs(cfg, anchors=anchors)
+    out, _ = _run(lib, inp)
+    _check(out, _ref(inp), cfg.W)
+
+
+def test_branch_dominant(lib):
+    # Branch keys scaled x4 (exact in bf16): their scores dominate the softmax,
+    # so any error in the branch tile, its mask or its RoPE shows at full size.
+    # Scaling the keys by 4 also scales the score error from rounding the
+    # rotated keys to bf16 (2^-9 relative) by 4, so this case gets 4x the
+    # unit-scale relative bound on its (now ~2.5-sized) outputs.
+    cfg = synth.custom_attn_config(1, (900,), 12, 8, 8, 2, 128, "bf16", seed=11)
+    inp = synth.attention_inputs(cfg)
+    k_br = inp.k_br * 4.0
+    out, _ = _run(lib, inp, k_br=k_br)
+    ref = _ref(inp, k_br=k_br)
+    got = to_np(out)
+    allr = np.concatenate([ref[b] for b in range(cfg.B)])
+    scale = np.max(np.abs(allr))
+    assert scale > 0.5  # the branch keys do carry the result
+    assert np.all(np.isfinite(got))
+    assert rel_err(got, allr) < 4 * RTOL
+
+
+def test_masked_keys_bit_invariant(lib):
+    # Changing trunk K/V after every anchor of the tile group, and the K/V of
+    # sibling branches, leaves the rows of branch 0 bit-identical.
+    cfg = synth.custom_attn_config(1, (600,), 8, 5, 8, 2, 128, "bf16", seed=5)
+    inp = synth.attention_inputs(cfg, anchors=[100, 120, 130, 200, 300, 400, 500, 590])
+    base, _ = _run(lib, inp)
+    k_tr = inp.k_tr.copy()
+    v_tr = inp.v_tr.copy()
+    k_tr[101:] = synth.round_bf16(k_tr[101:] * -3.0)
+    v_tr[101:] = synth.round_bf16(v_tr[101:] + 5.0)
+    out2, _ = _run(lib, inp, k_tr=k_tr, v_tr=v_tr)
+    rows0 = slice(0, cfg.W - 1)
+    assert torch.equal(out2[rows0], base[rows0])
+    assert not torch.equal(out2[cfg.W - 1:], base[cfg.W - 1:])
+
+
+def test_lse_bf16(lib):
+    cfg = synth.custom_attn_config(1, (400,), 4, 3, 4, 1, 128, "bf16", seed=2)
+    inp = synth.attention_inputs(cfg)
+    _, lse = _run(lib, inp, lse=True)
+    lse = to_np(lse)
+    # lse of one row from the oracle's rotated vectors
+    b, i, h = 1, 2, 3
+    r = b * (cfg.W - 1) + (i - 1)
+    a = int(inp.anchors[b])
+    pos = np.arange(a + cfg.W)
+    seq_k = np.concatenate([inp.k_tr[: a + 1], inp.k_br[b * (cfg.W - 1): (b + 1) * (cfg.W - 1)]])
+    k = oatt.rope(seq_k.astype(np.float64), pos, 1e4)[: a + 1 + i, 0]
+    q = oatt.rope(inp.q_br[r: r + 1].astype(np.float64), [a + i], 1e4)[0, h]
+    s = k @ q / np.sqrt(cfg.D)
+    ref = np.log(np.sum(np.exp(s - s.max()))) + s.max()
+    assert abs(lse[r, h] - ref) < 2e-2
+
+
+def test_anchor_out_of_range_bf16(lib):
+    cfg = synth.custom_attn_config(1, (256,), 3, 3, 8, 2, 128, "bf16", seed=9)
+    inp = synth.attention_inputs(cfg, anchors=[10, 300, 20])
+    out, _ = _run(lib, inp)
+    got = to_np(out)
+    assert np.all(np.isnan(got[2:4])) and np.all(np.isfinite(got[:2])) and np.all(np.isfinite(got[4:]))
+    assert lib.specopd_get_device_status() & lib.DEV_ANCHOR_RANGE
+
+
+@pytest.mark.parametrize("name,nsample", [("8b", None), ("long", 6), ("packed", 6)])
+def test_full_size_workloads(lib, name, nsample):
+    # The full workloads, in the launch configuration the benchmark times;
+    # the oracle checks every branch of the 8B shape and a seeded sample of
+    # branches of the long-trunk and packed workloads.
+    cfg = synth.attn_config(name)
+    inp = synth.attention_inputs(cfg)
+    out, _ = _run(lib, inp)
+    nb = cfg.S * cfg.B
+    if nsample is None:
+        branches = list(range(nb))
+    else:
+        rng = np.random.default_rng(123)
+        branches = sorted(set(rng.choice(nb, size=nsample, replace=False).tolist()) | {0, nb - 1})
+    _check(out, _ref(inp, branches=branches), cfg.W)
+    got = to_np(out)
+    assert np.all(np.isfinite(got))
+    assert lib.specopd_get_device_status() == 0

@@ -1,0 +1,63 @@
+// Internal launchers of the SpecOPD B200 library (host side, C++ linkage).
+// The exported C ABI lives in api.cu; these are the per-kernel launch
+// routines it dispatches to after validating arguments.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/specopd.h"
+
+namespace specopd {
+
+constexpr int kMaxSeq = 1024;  // sequences per call (cu_trunk travels as a kernel parameter)
+
+struct CuTrunk {
+  int S;
+  int T_tot;
+  int T_max;
+  int cu[kMaxSeq + 1];
+};
+
+// ---- tree build
+cudaError_t launch_tree_build(const CuTrunk& cu, const int32_t* anchors, int B, int W,
+                              int32_t* parent, int32_t* sem_pos, int32_t* score_row,
+                              cudaStream_t st);
+
+// ---- RoPE: y[t,h,:] = rope(x[t,h,:], pos[t]) for t < n (x may equal y).
+// theta: host array of D/2 frequencies base^(-2k/D) in double precision.
+cudaError_t launch_rope(specopd_dtype dt, const void* x, void* y, const int32_t* pos, int n, int H,
+                        int D, const double* theta_host, cudaStream_t st);
+
+// ---- tree attention, SIMT (fp32 workloads)
+struct AttnProblem {
+  int S, B, W, Hq, Hkv, D, G, R, T_tot, T_max;
+  float scale;  // softmax scale
+  specopd_dtype dtype;
+};
+cudaError_t launch_attn_simt_f32(const AttnProblem& p, const float* q_rot, const float* k_rot,
+                                 const float* v_br, const float* k_tr, const float* v_tr,
+                                 const int32_t* cu_trunk, const int32_t* anchors, float* out,
+                                 float* lse, cudaStream_t st);
+
+// ---- tree attention, tcgen05/TMEM/TMA (bf16 workloads)
+size_t attn_sm100_workspace(const AttnProblem& p);
+cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_rot, const void* k_rot,
+                              const void* v_br, const void* k_tr, const void* v_tr,
+                              const int32_t* cu_trunk, const int32_t* anchors, void* out,
+                              float* lse, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// ---- E2E-TV
+struct TVProblem {
+  int nbranch, W, V, N, rows_target;
+  specopd_dtype logit_dtype, grad_dtype;
+  int compute_grad;
+  double norm_count;
+};
+size_t tv_workspace(const TVProblem& p);
+cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_t* target_row,
+                          const void* z_draft, float* a, float* prefix, float* loss, double* numer,
+                          void* grad, void* ws, size_t ws_bytes, cudaStream_t st);
+
+}  // namespace specopd

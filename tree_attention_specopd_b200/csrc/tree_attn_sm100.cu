@@ -1,0 +1,656 @@
+// Tree-masked GQA attention of branch rows, bf16, tcgen05 / TMEM / TMA (sm_100a).
+//
+// SpecOPD review (jaehun.me) §3.2(a): the trunk K/V is computed once and
+// cached; the branch queries attach to that cache and each reads only itself
+// and its ancestors.  For branch row r = (s, b, i) the visible keys are the
+// trunk positions 0..a_b of sequence s and the branch nodes (s, b, 1..i);
+// siblings and later trunk tokens are masked.  Review §3.1: the condition of
+// position i is (x_{<=a_b}, y_{b,<i}).
+//
+// Tensor-core formulation (B200):
+//  * A work unit is (query tile, kv head, key chunk).  A query tile stacks
+//    RT = floor(128 / G) consecutive branch rows of one sequence times the G
+//    query heads of one kv head: M = RT*G <= 128 rows of the MMA.  The rows
+//    of a tile have nearby anchors (anchors are sorted per sequence), so the
+//    trunk keys a tile needs are [0, max anchor]; whole 128-key tiles beyond
+//    the tile's largest anchor are never loaded (masked-tile skipping), and
+//    each row masks only the ragged end of the last tile.
+//  * The branch keys are the tile's own branch nodes (plus the earlier nodes
+//    of its first branch): one or two extra 128-key tiles with the per-row
+//    mask first(branch) <= node <= row.  No dense T x T mask exists anywhere.
+//  * Long trunks are split into key chunks over several CTAs (split-KV);
+//    partial (O, max, sum) go to the workspace and the last CTA of a tile to
+//    finish merges them in a fixed order (no spin-wait, deterministic).
+//  * Per unit, warp 0 drives TMA (Q once, then K/V tiles in a 2-stage ring,
+//    128-byte swizzle), warp 1 issues tcgen05.mma from one thread:
+//    S = Q K^T into TMEM (two S buffers, so QK^T of tile j+1 overlaps the
+//    softmax of tile j), and O += P V with P read from TMEM (P overwrites
+//    its S buffer as bf16).  Warps 2-5 own one TMEM lane (= one query row)
+//    each: tcgen05.ld of the S row, mask, online softmax in the log2 domain
+//    with a lazy rescale (O is rescaled in TMEM only when the running max
+//    grows by more than 2^8), tcgen05.st of P.  The epilogue reads O from
+//    TMEM.
+//  * Every wait is bounded (%globaltimer); expiry sets the status word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace specopd {
+namespace sm100 {
+
+constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2..5: softmax
+constexpr int kBN = 128;       // keys per tile
+constexpr int kStages = 2;     // K and V ring depth
+constexpr int kTmemCols = 512;
+constexpr int kHalfBytes = 128 * 128;  // one [128 rows x 64 bf16] swizzled box
+constexpr float kRescaleThreshold = 8.f;  // log2 units
+
+struct Params {
+  int S, B, W, Hq, Hkv, G, R;
+  int RT;              // branch rows per query tile
+  int ntile_per_seq, ntile;
+  int nsplit, C;       // key chunks per (tile, kv head), keys per chunk (multiple of 128)
+  float scale_log2;    // softmax scale * log2(e)
+  const int32_t* cu_trunk;
+  const int32_t* anchors;
+  __nv_bfloat16* out;
+  float* lse;
+  float* part;         // split-KV partials
+  unsigned* cnt;       // [ntile * Hkv] arrival counters
+};
+
+struct Hdr {
+  uint64_t q_full;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_done;   // one phase per P.V tile (used by the lazy rescale)
+  uint64_t o_final;  // single phase: every MMA of the unit has completed
+  uint32_t tmem_base;
+  int kmax;
+  int last;
+  int abort;
+};
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+#define SPECOPD_R32(r)                                                                       \
+  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),        \
+      "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), \
+      "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),           \
+      "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),           \
+      "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define SPECOPD_W32(r)                                                                      \
+  "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),    \
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),       \
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),     \
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),     \
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+
+// 32 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : SPECOPD_R32(r)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};" ::"r"(taddr),
+      SPECOPD_W32(r)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100
+// version bits = 1.  lbo/sbo in bytes.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int N, bool b_mn_major) {
+  return (1u << 4)                      // D format f32
+         | (1u << 7)                    // A format bf16
+         | (1u << 10)                   // B format bf16
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, Hdr* hdr) {
+  if (mbar_wait(bar, parity)) return true;
+  hdr->abort = 1;
+  return false;
+}
+
+// Same, for the softmax warps: the result is uniform over the warp, because
+// the tcgen05.ld/st that follow are warp-collective (.sync.aligned).
+__device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, unsigned parity, Hdr* hdr) {
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity));
+  if (!ok) hdr->abort = 1;
+  return ok;
+}
+
+// ------------------------------------------------------------------ kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ktr,
+                 const __grid_constant__ CUtensorMap tm_vtr,
+                 const __grid_constant__ CUtensorMap tm_kbr,
+                 const __grid_constant__ CUtensorMap tm_vbr, const Params P) {
+  constexpr int NH = D / 64;     // 64-column halves of a row
+  constexpr int KSTEPS = D / 16; // MMA K steps of QK^T
+  extern __shared__ unsigned char smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sK = sQ + NH * kHalfBytes;
+  uint8_t* sV = sK + kStages * NH * kHalfBytes;
+  Hdr* hdr = reinterpret_cast<Hdr*>(sV + kStages * NH * kHalfBytes);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  // ---- work unit: (query tile, kv head, key chunk); heavier tiles first
+  const int u = blockIdx.x;
+  const int per_tile = P.Hkv * P.nsplit;
+  const int tile = P.ntile - 1 - u / per_tile;
+  const int c = (u % per_tile) / P.Hkv;
+  const int h = (u % per_tile) % P.Hkv;
+  const int s = tile / P.ntile_per_seq;
+  const int Wm1 = P.W - 1;
+  const int rows_seq = P.B * Wm1;
+  const int r0 = s * rows_seq + (tile % P.ntile_per_seq) * P.RT;
+  const int r1 = min(r0 + P.RT, (s + 1) * rows_seq);
+  const int t0 = P.cu_trunk[s];
+  const int Ts = P.cu_trunk[s + 1] - t0;
+
+  if (tid == 0) hdr->kmax = -1;
+  __syncthreads();
+  for (int r = r0 + tid; r < r1; r += kThreads) {
+    const int a = P.anchors[r / Wm1];
+    if (a >= 0 && a < Ts) atomicMax(&hdr->kmax, a);
+  }
+  __syncthreads();
+  const int kmax = hdr->kmax;
+  const int nact = kmax < 0 ? 1 : (kmax + P.C) / P.C;  // chunks with trunk keys (>= 1)
+  const int k_begin = c * P.C;
+  const int k_end = min(k_begin + P.C, kmax + 1);
+  const int nt = k_end > k_begin ? (k_end - k_begin + kBN - 1) / kBN : 0;
+  if (c > 0 && nt == 0) return;  // nothing for this chunk (uniform over the CTA)
+  const int kb0 = (r0 / Wm1) * Wm1;  // first branch node the tile needs
+  const int nbt = (c == 0) ? (r1 - kb0 + kBN - 1) / kBN : 0;
+  const int nk = nt + nbt;
+
+  // ---- barriers, TMEM
+  if (tid == 0) {
+    mbar_init(&hdr->q_full, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&hdr->k_full[i], 1);
+      mbar_init(&hdr->k_empty[i], 1);
+      mbar_init(&hdr->v_full[i], 1);
+      mbar_init(&hdr->v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&hdr->s_full[i], 1);
+      mbar_init(&hdr->p_full[i], 128);
+    }
+    mbar_init(&hdr->o_done, 1);
+    mbar_init(&hdr->o_final, 1);
+    hdr->abort = 0;
+    fence_mbar_init();
+  }
+  // Q rows beyond the tile (M = RT*G < 128) are never written by TMA: zero them.
+  const int MT = P.RT * P.G;
+  for (int idx = tid; idx < NH * (128 - MT) * 8; idx += kThreads) {
+    const int hh = idx / ((128 - MT) * 8);
+    const int rem = idx % ((128 - MT) * 8);
+    reinterpret_cast<uint4*>(sQ + hh * kHalfBytes + (MT + rem / 8) * 128)[rem % 8] =
+        make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&hdr->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = hdr->tmem_base;
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO = tmem + 256;
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const int G = P.G;
+      mbar_arrive_expect_tx(&hdr->q_full, (unsigned)(NH * MT * 128));
+      for (int hh = 0; hh < NH; ++hh)
+        tma_load_3d(sQ + hh * kHalfBytes, &tm_q, hh * 64, h * G, r0, &hdr->q_full);
+      for (int j = 0; j < nk && !hdr->abort; ++j) {
+        const int st = j % kStages;
+        const bool trunk = j < nt;
+        const int row = trunk ? t0 + k_begin + j * kBN : kb0 + (j - nt) * kBN;
+        if (j >= kStages && !wait_or_abort(&hdr->k_empty[st], ((j / kStages) - 1) & 1, hdr)) break;
+        mbar_arrive_expect_tx(&hdr->k_full[st], NH * kHalfBytes);
+        for (int hh = 0; hh < NH; ++hh)
+          tma_load_3d(sK + (st * NH + hh) * kHalfBytes, trunk ? &tm_ktr : &tm_kbr, hh * 64, h,
+                      row, &hdr->k_full[st]);
+        if (j >= kStages && !wait_or_abort(&hdr->v_empty[st], ((j / kStages) - 1) & 1, hdr)) break;
+        mbar_arrive_expect_tx(&hdr->v_full[st], NH * kHalfBytes);
+        for (int hh = 0; hh < NH; ++hh)
+          tma_load_3d(sV + (st * NH + hh) * kHalfBytes, trunk ? &tm_vtr : &tm_vbr, hh * 64, h,
+                      row, &hdr->v_full[st]);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdQK = idesc_bf16(kBN, false);
+      constexpr uint32_t kIdPV = idesc_bf16(D, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t k_addr = smem_u32(sK);
+      const uint32_t v_addr = smem_u32(sV);
+      auto pv = [&](int jj) -> bool {
+        const int b = jj & 1;
+        const int st = jj % kStages;
+        if (!wait_or_abort(&hdr->p_full[b], (jj >> 1) & 1, hdr)) return false;
+        if (!wait_or_abort(&hdr->v_full[st], (jj / kStages) & 1, hdr)) return false;
+        tc_fence_after();
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // B = V tile, MN-major: 16 keys = two 8-row groups of 1024 B; the
+          // 64-column halves of D are kHalfBytes apart.
+          const uint64_t bd = sdesc(v_addr + st * NH * kHalfBytes + kk * 2048, kHalfBytes, 1024);
+          mma_ts(tO, tS[b] + kk * 8, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&hdr->v_empty[st]);
+        tc_commit(&hdr->o_done);
+        return true;
+      };
+      bool ok = wait_or_abort(&hdr->q_full, 0, hdr);
+      tc_fence_after();
+      for (int j = 0; j < nk && ok; ++j) {
+        const int st = j % kStages;
+        const int b = j & 1;
+        if (!wait_or_abort(&hdr->k_full[st], (j / kStages) & 1, hdr)) { ok = false; break; }
+        tc_fence_after();
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          // K-major operands: 16 columns = 32 B inside a 128-byte swizzled row.
+          const int hh = kk >> 2, w = kk & 3;
+          const uint64_t ad = sdesc(q_addr + hh * kHalfBytes + w * 32, 16, 1024);
+          const uint64_t bd = sdesc(k_addr + (st * NH + hh) * kHalfBytes + w * 32, 16, 1024);
+          mma_ss(tS[b], ad, bd, kIdQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&hdr->k_empty[st]);
+        tc_commit(&hdr->s_full[b]);
+        if (j >= 1 && !pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && nk > 0) pv(nk - 1);
+      // A commit tracks every MMA issued before it: the epilogue waits on this
+      // one barrier instead of a phase of o_done, which can be two phases
+      // behind there (P.V of tile nk-2 is issued after the last S commit).
+      tc_commit(&hdr->o_final);
+    }
+  } else {
+    // ================================================================ softmax / epilogue
+    const int q4 = warp & 3;             // TMEM lane quadrant of this warp
+    const int mrow = q4 * 32 + lane;     // query row of the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const int G = P.G;
+    const int lr = mrow / G, g = mrow % G;
+    const int r = r0 + lr;
+    const bool in_tile = (lr < P.RT) && (r < r1);
+    int a_r = -1, kfirst = 0;
+    bool bad = false;
+    if (in_tile) {
+      const int bid = r / Wm1;
+      a_r = P.anchors[bid];
+      bad = (a_r < 0 || a_r >= Ts);
+      kfirst = bid * Wm1;
+    }
+    const bool live = in_tile && !bad;
+    const float sl2 = P.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    uint32_t sv[kBN];
+    for (int j = 0; j < nk; ++j) {
+      const int b = j & 1;
+      if (!warp_wait_or_abort(&hdr->s_full[b], (j >> 1) & 1, hdr)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < kBN / 32; ++q) tmem_ld32(tS[b] + lane_off + q * 32, sv + q * 32);
+      tmem_wait_ld();
+      // visible columns: lo <= col <= hi
+      int lo, hi;
+      if (j < nt) {
+        lo = 0;
+        hi = a_r - (k_begin + j * kBN);
+      } else {
+        const int node0 = kb0 + (j - nt) * kBN;
+        lo = kfirst - node0;
+        hi = r - node0;
+      }
+      if (!live) hi = -1;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int col = 0; col < kBN; ++col) {
+        const float x = (col >= lo && col <= hi) ? __uint_as_float(sv[col]) * sl2 : -INFINITY;
+        sv[col] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      const float m_new = fmaxf(m, mx);
+      // Lazy rescale: keep the stale max unless it grew by more than 2^8.
+      const bool need = (m != -INFINITY) && (m_new > m + kRescaleThreshold);
+      if (m == -INFINITY) m = m_new;  // first visible keys: O and l are still zero
+      if (__any_sync(0xffffffffu, need)) {
+        // Warp-uniform branch (the TMEM accesses are warp-collective); rows
+        // that need no rescale multiply by 1.
+        const float f = need ? exp2f(m - m_new) : 1.f;
+        if (need) {
+          l *= f;
+          m = m_new;
+        }
+        if (j > 0) {
+          // O holds PV of tiles < j; PV of tile j-1 must be complete.
+          if (!warp_wait_or_abort(&hdr->o_done, (j - 1) & 1, hdr)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t ov[32];
+            tmem_ld32(tO + lane_off + q * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+            tmem_st32(tO + lane_off + q * 32, ov);
+          }
+        }
+      }
+      float rs = 0.f;
+      uint32_t pk[kBN / 2];
+#pragma unroll
+      for (int e = 0; e < kBN / 2; ++e) {
+        const float x0 = __uint_as_float(sv[2 * e]);
+        const float x1 = __uint_as_float(sv[2 * e + 1]);
+        const float p0 = (m == -INFINITY) ? 0.f : exp2f(x0 - m);
+        const float p1 = (m == -INFINITY) ? 0.f : exp2f(x1 - m);
+        rs += p0 + p1;
+        pk[e] = pack_bf16x2(p0, p1);
+      }
+      l += rs;
+      tmem_st32(tS[b] + lane_off, pk);
+      tmem_st32(tS[b] + lane_off + 32, pk + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&hdr->p_full[b]);
+    }
+    // ---- epilogue
+    float o[D];
+    const bool ok = warp_wait_or_abort(&hdr->o_final, 0, hdr) && !hdr->abort;
+    tc_fence_after();
+#pragma unroll
+    for (int q = 0; q < D / 32; ++q) {
+      uint32_t ov[32];
+      tmem_ld32(tO + lane_off + q * 32, ov);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[q * 32 + e] = __uint_as_float(ov[e]);
+    }
+    const int hq = h * G + g;
+    const float qnan = __int_as_float(0x7fc00000);
+    auto write_row = [&](const float* acc, float mm, float ll) {
+      __nv_bfloat16* dst = P.out + ((size_t)r * P.Hq + hq) * D;
+      const float inv = (bad || !ok) ? qnan : 1.f / ll;
+#pragma unroll
+      for (int e = 0; e < D; e += 8) {
+        uint4 v;
+        v.x = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+        v.y = pack_bf16x2(acc[e + 2] * inv, acc[e + 3] * inv);
+        v.z = pack_bf16x2(acc[e + 4] * inv, acc[e + 5] * inv);
+        v.w = pack_bf16x2(acc[e + 6] * inv, acc[e + 7] * inv);
+        *reinterpret_cast<uint4*>(dst + e) = v;
+      }
+      if (P.lse) P.lse[(size_t)r * P.Hq + hq] = (bad || !ok) ? qnan : (mm + log2f(ll)) * 0.6931471805599453f;
+      if (bad && g == 0) set_status(SPECOPD_DEV_ANCHOR_RANGE);
+    };
+    if (nact == 1) {
+      if (in_tile) write_row(o, m, l);
+    } else {
+      // split-KV: publish this chunk's partial, the last chunk to arrive merges
+      const size_t slot = ((size_t)tile * P.Hkv + h) * P.nsplit;
+      const size_t slot_floats = (size_t)128 * D + 256;
+      float* mine = P.part + (slot + c) * slot_floats;
+#pragma unroll
+      for (int e = 0; e < D; e += 4)
+        __stcg(reinterpret_cast<float4*>(mine + (size_t)mrow * D + e),
+               make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
+      mine[128 * D + mrow] = m;
+      mine[128 * D + 128 + mrow] = l;
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (mrow == 0) {
+        const unsigned old = atomicAdd(&P.cnt[tile * P.Hkv + h], 1u);
+        hdr->last = (old == (unsigned)nact - 1u) ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (hdr->last) {
+        __threadfence();
+        float mm = -INFINITY;
+        for (int cc = 0; cc < nact; ++cc)
+          mm = fmaxf(mm, __ldcg(P.part + (slot + cc) * slot_floats + 128 * D + mrow));
+        float ll = 0.f;
+#pragma unroll
+        for (int e = 0; e < D; ++e) o[e] = 0.f;
+        for (int cc = 0; cc < nact; ++cc) {
+          const float* pc = P.part + (slot + cc) * slot_floats;
+          const float mc = __ldcg(pc + 128 * D + mrow);
+          const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - mm);
+          ll += wgt * __ldcg(pc + 128 * D + 128 + mrow);
+#pragma unroll
+          for (int e = 0; e < D; e += 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(pc + (size_t)mrow * D + e));
+            o[e] += wgt * v.x;
+            o[e + 1] += wgt * v.y;
+            o[e + 2] += wgt * v.z;
+            o[e + 3] += wgt * v.w;
+          }
+        }
+        if (in_tile) write_row(o, mm, ll);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D view [rows, H, D] (bf16, contiguous) with box (64, box_h, box_rows).
+bool make_map(CUtensorMap* m, const void* ptr, int D, int H, int rows, int box_h, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_h, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Plan {
+  int RT, ntile_per_seq, ntile, nsplit, C;
+  size_t part_bytes, cnt_bytes;
+};
+
+Plan make_plan(const AttnProblem& p) {
+  Plan pl;
+  pl.RT = 128 / p.G;
+  const int rows_seq = p.B * (p.W - 1);
+  pl.ntile_per_seq = (rows_seq + pl.RT - 1) / pl.RT;
+  pl.ntile = pl.ntile_per_seq * p.S;
+  const long long base = (long long)pl.ntile * p.Hkv;
+  int nsplit = 1;
+  if (base < 2 * 148) {
+    nsplit = (int)((2 * 148 + base - 1) / base);
+    const int max_split = std::max(1, p.T_max / 512);
+    if (nsplit > max_split) nsplit = max_split;
+  }
+  int C = (p.T_max + nsplit - 1) / nsplit;
+  C = (C + kBN - 1) / kBN * kBN;
+  nsplit = (p.T_max + C - 1) / C;
+  pl.nsplit = nsplit;
+  pl.C = C;
+  pl.part_bytes = nsplit > 1 ? (size_t)pl.ntile * p.Hkv * nsplit * ((size_t)128 * p.D + 256) * 4 : 0;
+  pl.cnt_bytes = (size_t)pl.ntile * p.Hkv * 4;
+  return pl;
+}
+
+size_t smem_bytes(int D) {
+  const int NH = D / 64;
+  size_t b = 1024 + (size_t)NH * kHalfBytes * (1 + 2 * kStages) + sizeof(Hdr);
+  // D = 64 would fit two CTAs per SM; each allocates all 512 TMEM columns, so
+  // keep one CTA per SM.
+  if (b < 120 * 1024) b = 120 * 1024;
+  return b;
+}
+
+}  // namespace
+}  // namespace sm100
+
+size_t attn_sm100_workspace(const AttnProblem& p) {
+  const sm100::Plan pl = sm100::make_plan(p);
+  return ((pl.part_bytes + 255) & ~size_t(255)) + pl.cnt_bytes;
+}
+
+cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_rot, const void* k_rot,
+                              const void* v_br, const void* k_tr, const void* v_tr,
+                              const int32_t* cu_trunk, const int32_t* anchors, void* out,
+                              float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+  using namespace sm100;
+  if (p.R == 0) return cudaSuccess;
+  if (p.D != 64 && p.D != 128) return cudaErrorInvalidValue;
+  const Plan pl = make_plan(p);
+  const size_t part_off = 0;
+  const size_t cnt_off = (pl.part_bytes + 255) & ~size_t(255);
+  if (ws_bytes < cnt_off + pl.cnt_bytes) return cudaErrorInvalidValue;
+  CUtensorMap tq, tktr, tvtr, tkbr, tvbr;
+  if (!make_map(&tq, q_rot, p.D, p.Hq, p.R, p.G, pl.RT) ||
+      !make_map(&tktr, k_tr, p.D, p.Hkv, p.T_tot, 1, kBN) ||
+      !make_map(&tvtr, v_tr, p.D, p.Hkv, p.T_tot, 1, kBN) ||
+      !make_map(&tkbr, k_rot, p.D, p.Hkv, p.R, 1, kBN) ||
+      !make_map(&tvbr, v_br, p.D, p.Hkv, p.R, 1, kBN))
+    return cudaErrorInvalidValue;
+  Params P;
+  P.S = p.S; P.B = p.B; P.W = p.W; P.Hq = p.Hq; P.Hkv = p.Hkv; P.G = p.G; P.R = p.R;
+  P.RT = pl.RT; P.ntile_per_seq = pl.ntile_per_seq; P.ntile = pl.ntile;
+  P.nsplit = pl.nsplit; P.C = pl.C;
+  P.scale_log2 = p.scale * 1.4426950408889634f;
+  P.cu_trunk = cu_trunk;
+  P.anchors = anchors;
+  P.out = reinterpret_cast<__nv_bfloat16*>(out);
+  P.lse = lse;
+  char* w = reinterpret_cast<char*>(ws);
+  P.part = reinterpret_cast<float*>(w + part_off);
+  P.cnt = reinterpret_cast<unsigned*>(w + cnt_off);
+  cudaError_t e = cudaMemsetAsync(w + cnt_off, 0, pl.cnt_bytes, st);
+  if (e != cudaSuccess) return e;
+  const size_t smem = smem_bytes(p.D);
+  const dim3 grid((unsigned)((size_t)pl.ntile * p.Hkv * pl.nsplit));
+  if (p.D == 128) {
+    e = cudaFuncSetAttribute(tree_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    tree_attn_kernel<128><<<grid, kThreads, smem, st>>>(tq, tktr, tvtr, tkbr, tvbr, P);
+  } else {
+    e = cudaFuncSetAttribute(tree_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    tree_attn_kernel<64><<<grid, kThreads, smem, st>>>(tq, tktr, tvtr, tkbr, tvbr, P);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace specopd
