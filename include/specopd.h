@@ -252,6 +252,37 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* desc,
                               float* loss, double* numer, void* grad_draft,
                               void* workspace, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* E2E-TV for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is an interface addition of this library.
+ *
+ * Some callers cannot call cudaMalloc: code that runs inside another
+ * framework's memory pool (which owns the device memory and forbids
+ * allocations outside it), or code on a path where cudaMalloc's implicit
+ * device-wide synchronisation is not allowed.  specopd_e2e_tv_noalloc
+ * computes exactly what specopd_e2e_tv computes (same arguments, minus the
+ * workspace) and allocates nothing: its scratch is a fixed array of
+ * SPECOPD_E2E_TV_STATIC_SCRATCH_BYTES in the library's device image, held by
+ * every GPU that loads the library until the process exits.
+ *   - Size limit: returns SPECOPD_ERR_WORKSPACE, launching nothing, when
+ *     specopd_e2e_tv_workspace_size(desc) exceeds the array (1 MiB holds
+ *     about 60,000 positions).
+ *   - The first call on each device resolves the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents (each call clears what must start at zero).  Calls that
+ *     overlap on the GPU -- other streams, other host threads -- race on it:
+ *     serialise them.
+ */
+#define SPECOPD_E2E_TV_STATIC_SCRATCH_BYTES (1u << 20)
+
+specopd_status specopd_e2e_tv_noalloc(const specopd_tv_desc* desc,
+                                      const void* z_target,
+                                      const int32_t* target_row,
+                                      const void* z_draft, float* a, float* prefix,
+                                      float* loss, double* numer, void* grad_draft,
+                                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -88,6 +88,9 @@ def load(path: str = LIB_PATH):
     lib.specopd_e2e_tv.restype = cint
     lib.specopd_e2e_tv.argtypes = [ctypes.POINTER(TVDesc), vp, i32p, vp, f32p, f32p, f32p,
                                    f64p, vp, vp, csize, vp]
+    lib.specopd_e2e_tv_noalloc.restype = cint
+    lib.specopd_e2e_tv_noalloc.argtypes = [ctypes.POINTER(TVDesc), vp, i32p, vp, f32p, f32p,
+                                           f32p, f64p, vp, vp]
     _lib = lib
     return lib
 
@@ -220,4 +223,20 @@ def specopd_e2e_tv(desc, z_target, target_row, z_draft, a=None, prefix=None, los
                                  _ptr(z_draft), _ptr(a), _ptr(prefix), _ptr(loss), _ptr(numer),
                                  _ptr(grad), _ptr(workspace), workspace.numel(), _stream(stream)),
            "e2e_tv")
+    return {"a": a, "prefix": prefix, "loss": loss, "numer": numer, "grad": grad}
+
+
+E2E_TV_STATIC_SCRATCH_BYTES = 1 << 20
+
+
+def specopd_e2e_tv_noalloc(desc, z_target, target_row, z_draft, a, prefix, loss, numer=None,
+                           grad=None, stream=None):
+    """E2E-TV without a workspace argument, for callers that cannot allocate
+    device memory (the library's fixed 1 MiB scratch array is used instead).
+    All outputs are caller-provided; calls that overlap on the GPU race on the
+    shared scratch and must be serialised."""
+    _check(load().specopd_e2e_tv_noalloc(ctypes.byref(desc), _ptr(z_target), _ptr(target_row),
+                                         _ptr(z_draft), _ptr(a), _ptr(prefix), _ptr(loss),
+                                         _ptr(numer), _ptr(grad), _stream(stream)),
+           "e2e_tv_noalloc")
     return {"a": a, "prefix": prefix, "loss": loss, "numer": numer, "grad": grad}

@@ -268,3 +268,6 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* d, const void* z_target,
 }
 
 }  // extern "C"
+
+// Entry point without a workspace argument (library-owned scratch).
+#include "e2e_tv_noalloc.cu"
