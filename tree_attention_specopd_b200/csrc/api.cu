@@ -114,7 +114,7 @@ specopd_status tv_problem(const specopd_tv_desc* d, TVProblem& p) {
   p.compute_grad = d->compute_grad ? 1 : 0;
   p.norm_count = d->norm_count > 0 ? (double)d->norm_count : (double)N;
   // Cluster size needed to hold both rows in shared memory (<= 16 CTAs).
-  const long long CL = (4ll * d->V * (long long)elt(d->logit_dtype) + kTVSmemBudget - 1) / kTVSmemBudget;
+  const long long CL = (2ll * kTVBuffers * d->V * (long long)elt(d->logit_dtype) + kTVSmemBudget - 1) / kTVSmemBudget;
   if (CL > 16) return SPECOPD_ERR_UNSUPPORTED;
   return SPECOPD_OK;
 }

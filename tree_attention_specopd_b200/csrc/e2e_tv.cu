@@ -18,27 +18,37 @@
 //
 // B200 design (HBM-bound: the algorithmic traffic is one read of both logit
 // rows and one write of the gradient):
-//  * One persistent launch of thread-block clusters.  Work is a queue of
-//    tasks claimed with one atomic per task:
-//      A(n): bulk-copy (TMA 1-D) the two logit rows of position n into the
-//            cluster's shared memory, each CTA holding a 1/CL slice; online
-//            max / sum-exp, a DSMEM reduction of the statistics, then the
-//            overlap a_n and s_n from shared memory (no second HBM read),
-//            another DSMEM reduction.  The A-task that completes a branch
-//            (atomic count) runs the branch's prefix scan and gradient
-//            coefficients; the one that completes the last branch reduces
-//            the loss in a fixed order (deterministic).
-//      G(n): wait (bounded) until branch b is scanned, stream the two rows
-//            again -- by queue construction they were read a few tasks ago
-//            and are still resident in the 126 MB L2 -- and write dz.
-//    G-tasks of branch b are queued `lag` branches after its A-tasks, and a
-//    G-task only ever waits for A-tasks claimed before it, which never wait:
-//    the queue cannot deadlock whatever the residency of the grid.
+//  * One persistent launch of thread-block clusters of CL CTAs; each CTA
+//    owns a 1/CL slice of the vocabulary.  Work is a queue of tasks claimed
+//    with one atomic each, two tasks ahead so the atomic's latency hides
+//    behind the current task:
+//      A(n): the two logit rows of position n arrive by 1-D bulk copy (TMA)
+//            into shared memory; online max / sum-exp, a DSMEM reduction of
+//            the statistics over the cluster, the overlap a_n and s_n from
+//            shared memory, a second DSMEM reduction; publish (lse, s, a)
+//            and count the branch (release, fire-and-forget).
+//      G(n): wait (bounded) until all W positions of branch b are counted,
+//            load the branch's W overlaps in one parallel read, form g_n,
+//            and write dz from the rows, which were copied in (from L2:
+//            the A-task read them a few tasks earlier) during the previous
+//            task.  G(b, 1) also writes the branch's prefix products and
+//            adds the branch to the loss.
+//      S(b): (no gradient requested) the prefix products and loss part of
+//            G(b, 1) alone.
+//    Each CTA double-buffers its shared memory: the next task's bulk copies
+//    stream in while the current task computes.  G/S tasks of branch b are
+//    queued `lag` branches after its A-tasks, and only ever wait for
+//    A-tasks, which never wait and were claimed earlier: the lowest
+//    unfinished task is always running, so the queue cannot deadlock
+//    whatever the residency of the grid.
+//  * The loss is reduced by the last branch to finish, in a fixed order:
+//    deterministic.
 //  * All math in the log2 domain: x2 = z*log2(e) - lse2 via one FMA, one
 //    ex2 per element per pass.  The same FMA sequence decides [q < p] in the
 //    A- and the G-task, so s_n and the gradient's mask always agree.
 #include <cooperative_groups.h>
 
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -50,11 +60,16 @@ namespace cg = cooperative_groups;
 
 namespace specopd {
 
-constexpr int kTVThreads = 512;
+constexpr int kTVThreads = 256;
 constexpr int kTVWarps = kTVThreads / 32;
-constexpr int kTVChunks = 4;            // bulk copies per row slice (pipelined)
-constexpr int kTVSmemBudget = 210 * 1024;  // bytes of row slices per CTA (2 tasks)
+constexpr int kTVCtasPerSm = 2;            // independent CTAs per SM hide each other's waits
+constexpr int kTVBuffers = 1;              // row-slice buffers per CTA
+constexpr int kTVChunks = 4;               // bulk copies per row slice (pipelined)
+constexpr int kTVSmemBudget = 104 * 1024;  // bytes of row slices per CTA
+constexpr int kTVMaxW = 1024;              // positions per branch held in shared memory
 constexpr float kLog2e = 1.4426950408889634f;
+
+enum TaskKind { kTaskA = 0, kTaskG = 1, kTaskS = 2 };
 
 struct TVArgs {
   int nbranch, W, V, N, rows_target, compute_grad;
@@ -69,30 +84,37 @@ struct TVArgs {
   float* loss;
   double* numer;
   void* grad;
-  float4* rec;       // [N]  (lse2_t, lse2_d, s, g)
+  float4* rec;       // [N]  (lse2_t, lse2_d, s, unused)
   double* bsum;      // [nbranch]
-  unsigned* cnt;     // [nbranch]
-  unsigned* ready;   // [nbranch]
+  unsigned* cnt;     // [nbranch] positions of the branch published
   unsigned* ctl;     // [0] claim, [1] branches done, [2] abort
 };
 
-// Task id -> (is_A, position).  See the queue description above.
-__device__ __forceinline__ void decode_task(const TVArgs& A, int t, bool& isA, int& pos) {
+// Task id -> (kind, index).  index = position for A and G, branch for S.
+// Queue: slot k holds the W A-tasks of branch k, then the second-kind tasks
+// (W G-tasks, or one S-task) of branch k - lag.
+__device__ __forceinline__ void decode_task(const TVArgs& A, int t, int& kind, int& idx) {
   const int W = A.W;
-  if (!A.compute_grad) { isA = true; pos = t; return; }
+  const int per = A.compute_grad ? W : 1;
   const int k0 = min(A.lag, A.nbranch);
-  if (t < k0 * W) { isA = true; pos = t; return; }
+  if (t < k0 * W) { kind = kTaskA; idx = t; return; }
   const int t1 = t - k0 * W;
   const int n_mid = max(0, A.nbranch - A.lag);
-  if (t1 < n_mid * 2 * W) {
-    const int k = A.lag + t1 / (2 * W);
-    const int w = t1 % (2 * W);
-    if (w < W) { isA = true; pos = k * W + w; }
-    else { isA = false; pos = (k - A.lag) * W + (w - W); }
-    return;
+  const int blk = W + per;
+  int b2, j2;
+  if (t1 < n_mid * blk) {
+    const int k = A.lag + t1 / blk;
+    const int w = t1 % blk;
+    if (w < W) { kind = kTaskA; idx = k * W + w; return; }
+    b2 = k - A.lag;
+    j2 = w - W;
+  } else {
+    const int t2 = t1 - n_mid * blk;
+    b2 = n_mid + t2 / per;
+    j2 = t2 % per;
   }
-  isA = false;
-  pos = n_mid * W + (t1 - n_mid * 2 * W);
+  if (A.compute_grad) { kind = kTaskG; idx = b2 * W + j2; }
+  else { kind = kTaskS; idx = b2; }
 }
 
 template <typename Tin> struct Vec;
@@ -102,6 +124,15 @@ template <> struct Vec<__nv_bfloat16> {
     f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
     f[4] = bf16lo(u.z); f[5] = bf16hi(u.z); f[6] = bf16lo(u.w); f[7] = bf16hi(u.w);
   }
+  // max of the 8 values, with packed bf16x2 comparisons
+  static __device__ __forceinline__ float vmax(const uint4& u) {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162*>(&u.z);
+    const __nv_bfloat162 d = *reinterpret_cast<const __nv_bfloat162*>(&u.w);
+    const __nv_bfloat162 m = __hmax2(__hmax2(a, b), __hmax2(c, d));
+    return fmaxf(__low2float(m), __high2float(m));
+  }
 };
 template <> struct Vec<float> {
   static constexpr int kN = 4;
@@ -109,80 +140,51 @@ template <> struct Vec<float> {
     f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
     f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
   }
+  static __device__ __forceinline__ float vmax(const uint4& u) {
+    return fmaxf(fmaxf(__uint_as_float(u.x), __uint_as_float(u.y)),
+                 fmaxf(__uint_as_float(u.z), __uint_as_float(u.w)));
+  }
 };
 
-// Online (max, sum 2^(x - max)) over a group of values already in log2 units.
-template <int K>
-__device__ __forceinline__ void online_update(float& m, float& s, const float* x2) {
-  float mx = x2[0];
-#pragma unroll
-  for (int k = 1; k < K; ++k) mx = fmaxf(mx, x2[k]);
-  const float mn = fmaxf(m, mx);
-  if (mn == -INFINITY) return;
-  float acc = (m == -INFINITY) ? 0.f : s * exp2f(m - mn);
-#pragma unroll
-  for (int k = 0; k < K; ++k) acc += exp2f(x2[k] - mn);
-  m = mn;
-  s = acc;
-}
-
-// Block-wide combine of per-thread (m, s) pairs; result valid in all threads.
-__device__ __forceinline__ void block_lse2(float& m, float& s, float2* red /*[kTVWarps]*/) {
+__device__ __forceinline__ void warp_lse2(float& m, float& s) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
     const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
     lse2_combine(m, s, m2, s2);
   }
-  const int warp = threadIdx.x >> 5;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[warp] = make_float2(m, s);
-  __syncthreads();
-  m = -INFINITY; s = 0.f;
-  for (int w = 0; w < kTVWarps; ++w) lse2_combine(m, s, red[w].x, red[w].y);
 }
 
-__device__ __forceinline__ float block_sum(float v, float* red /*[kTVWarps]*/) {
-  v = warp_sum(v);
-  const int warp = threadIdx.x >> 5;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[warp] = v;
-  __syncthreads();
-  float t = 0.f;
-  for (int w = 0; w < kTVWarps; ++w) t += red[w];
-  return t;
+// Cluster barrier without a release by every thread: a release arrive would
+// make each thread drain its outstanding global stores (the gradient rows)
+// at every barrier.  All threads execute the same aligned instructions (the
+// barrier is never reached divergently); the one thread that wrote shared
+// memory another CTA reads after the barrier issues a cluster-scope fence
+// first (publish_for_cluster), and the wait is an acquire.
+__device__ __forceinline__ void publish_for_cluster() {
+  asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_barrier_relaxed() {
+  __syncwarp();  // the .aligned form needs a converged warp
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
 struct TVShared {
-  int task[2];      // claimed task ids, by iteration parity
+  int task[4];       // claimed task ids, ring indexed by iteration
   int flag;
-  int pad;
-  uint64_t bar[2][kTVChunks];  // bulk-copy completion, per buffer and chunk
-  float4 cl_red1;   // this CTA's (m_t, s_t, m_d, s_d) for the cluster reduction
-  float2 cl_red2;   // this CTA's (a, s) partial
-  float2 wred[kTVWarps];
-  float fred[kTVWarps];
-  float fred2[kTVWarps];
+  float g;           // gradient coefficient of the current G-task
+  uint64_t bar[kTVBuffers][kTVChunks];  // bulk-copy completion, per buffer and chunk
+  float4 red_lse[kTVWarps];    // per-warp (m_t, s_t, m_d, s_d)
+  float2 red_as[kTVWarps];     // per-warp (a, s)
+  float4 cl_lse;     // this CTA's statistics, read by the cluster
+  float2 cl_as;      // this CTA's (a, s), read by the cluster
+  float4 all_lse;    // cluster-combined statistics
   double dred[kTVWarps];
+  float sa[kTVMaxW];  // overlaps of one branch
 };
-
-// Row addresses of task t for this CTA's slice.
-struct TaskRows {
-  bool isA, row_ok;
-  int pos, b;
-};
-
-__device__ __forceinline__ TaskRows task_rows(const TVArgs& A, int t) {
-  TaskRows tr;
-  decode_task(A, t, tr.isA, tr.pos);
-  tr.b = tr.pos / A.W;
-  const int row = A.trow ? A.trow[tr.pos] : tr.pos;
-  tr.row_ok = (row >= 0 && row < A.rows_target);
-  return tr;
-}
 
 template <typename Tin, typename Tg>
-__global__ void __launch_bounds__(kTVThreads, 1) e2e_tv_kernel(const TVArgs A) {
+__global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const TVArgs A) {
   extern __shared__ __align__(128) unsigned char tv_smem_raw[];
   TVShared& sh = *reinterpret_cast<TVShared*>(tv_smem_raw);
   Tin* buf0 = reinterpret_cast<Tin*>(tv_smem_raw + ((sizeof(TVShared) + 127) / 128) * 128);
@@ -190,16 +192,18 @@ __global__ void __launch_bounds__(kTVThreads, 1) e2e_tv_kernel(const TVArgs A) {
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   constexpr int VN = Vec<Tin>::kN;
 
   if (tid == 0) {
-    for (int bb = 0; bb < 2; ++bb)
+    for (int bb = 0; bb < kTVBuffers; ++bb)
       for (int c = 0; c < kTVChunks; ++c) mbar_init(&sh.bar[bb][c], 1);
     fence_mbar_init();
   }
   __syncthreads();
 
   const int V = A.V;
+  const int W = A.W;
   const int v0 = rank * A.Lc;
   const int len = max(0, min(V, v0 + A.Lc) - v0);
   const int chunk_elems = ((A.Lc / kTVChunks) + 15) / 16 * 16;
@@ -212,16 +216,16 @@ __global__ void __launch_bounds__(kTVThreads, 1) e2e_tv_kernel(const TVArgs A) {
     rt = zt + (long long)row * V + v0;
     rd = zd + (long long)pos * V + v0;
   };
-  // Buffer bb holds the slices (st, sd) of one task: [Lc] target, [Lc] draft.
   auto buf_t = [&](int bb) { return buf0 + (size_t)bb * 2 * A.Lc; };
   auto buf_d = [&](int bb) { return buf0 + (size_t)bb * 2 * A.Lc + A.Lc; };
 
-  // Issue the asynchronous bulk copies of task t into buffer bb (aligned path).
+  // Start the bulk copies of task t's rows into buffer bb (aligned path; A and
+  // G tasks only -- S tasks touch no rows).
   auto issue_loads = [&](int t, int bb) {
     if (t >= A.total_tasks || !A.aligned || tid != 0) return;
-    bool isA;
-    int pos;
-    decode_task(A, t, isA, pos);
+    int kind, pos;
+    decode_task(A, t, kind, pos);
+    if (kind == kTaskS) return;
     const Tin *rt, *rd;
     row_ptrs(pos, rt, rd);
     Tin* st = buf_t(bb);
@@ -238,50 +242,121 @@ __global__ void __launch_bounds__(kTVThreads, 1) e2e_tv_kernel(const TVArgs A) {
       }
     }
   };
+  // Every A and G task uses its buffer once: buffer bb's k-th use waits for
+  // its barriers' phase k.
+  unsigned uses[kTVBuffers] = {};
 
-  auto claim = [&](int slot) {
-    if (rank == 0 && tid == 0) {
-      int t = A.total_tasks;
-      if (*((volatile unsigned*)&A.ctl[2]) == 0u) t = (int)atomicAdd(&A.ctl[0], 1u);
-      if (t > A.total_tasks) t = A.total_tasks;
-      for (int r = 0; r < A.CL; ++r) *cluster.map_shared_rank(&sh.task[slot], r) = t;
+  auto claim = [&]() -> int {
+    int t = A.total_tasks;
+    if (*((volatile unsigned*)&A.ctl[2]) == 0u) t = (int)atomicAdd(&A.ctl[0], 1u);
+    return t > A.total_tasks ? A.total_tasks : t;
+  };
+  auto broadcast = [&](int slot, int t) {
+    for (int r = 0; r < A.CL; ++r) *cluster.map_shared_rank(&sh.task[slot], r) = t;
+  };
+
+  // Loss of the last branch to finish: 1 - sum_b bsum[b] / norm, fixed order.
+  auto finish_loss = [&]() {
+    double acc = 0.0;
+    for (int i = tid; i < A.nbranch; i += kTVThreads) acc += __ldcg(&A.bsum[i]);
+    acc = warp_sum_d(acc);
+    if (lane == 0) sh.dred[warp] = acc;
+    __syncthreads();
+    if (tid == 0) {
+      double tot = 0.0;
+      for (int w = 0; w < kTVWarps; ++w) tot += sh.dred[w];
+      A.loss[0] = (float)(1.0 - tot / A.norm);
+      if (A.numer) A.numer[0] = tot;
     }
   };
 
-  claim(0);
-  cluster.sync();
-  issue_loads(sh.task[0], 0);
+  // Wait until branch b's W positions are published, then stage its overlaps
+  // in sh.sa (all threads of the CTA take part).  Returns false on timeout.
+  auto stage_branch = [&](int b) -> bool {
+    if (tid == 0) {
+      const bool ok = wait_flag_geq(&A.cnt[b], (unsigned)W);
+      if (!ok) atomicExch(&A.ctl[2], 1u);
+      sh.flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    const bool ok = sh.flag != 0;
+    if (ok)
+      for (int i = tid; i < W; i += kTVThreads) sh.sa[i] = __ldcg(&A.a_out[b * W + i]);
+    __syncthreads();
+    return ok;
+  };
+  // Prefix products of branch b from sh.sa; writes prefix[] and bsum[b] and
+  // counts the branch; the last branch reduces the loss.  Rank 0 only.
+  auto scan_branch = [&](int b) {
+    if (tid == 0) {
+      float P = 1.f;
+      double sumP = 0.0;
+      for (int i = 0; i < W; ++i) {
+        P *= sh.sa[i];
+        A.prefix[b * W + i] = P;
+        sumP += (double)P;
+      }
+      A.bsum[b] = sumP;
+      __threadfence();
+      const unsigned done = atomicAdd(&A.ctl[1], 1u);
+      sh.flag = (done == (unsigned)A.nbranch - 1u) ? 1 : 0;
+      if (sh.flag) __threadfence();
+    }
+    __syncthreads();
+    if (sh.flag) finish_loss();
+  };
+
+  if (rank == 0 && tid == 0) {
+    const int t0 = claim();
+    const int t1 = claim();
+    broadcast(0, t0);
+    broadcast(1, t1);
+    publish_for_cluster();
+  }
+  cluster_barrier_relaxed();
+  if (kTVBuffers == 2) issue_loads(sh.task[0], 0);
 
   for (int k = 0;; ++k) {
-    const int t = sh.task[k & 1];
+    const int t = sh.task[k & 3];
     if (t >= A.total_tasks) break;
-    // Claim the next task now and start its copies into the other buffer, so
-    // they stream while this task computes.  The cluster barrier also ends
-    // every thread's use of that buffer (task k-1).
-    claim((k + 1) & 1);
-    cluster.sync();
-    issue_loads(sh.task[(k + 1) & 1], (k + 1) & 1);
+    // Claim task k+2 now; its id is broadcast at the end of this task.
+    int t_ahead = A.total_tasks;
+    if (rank == 0 && tid == 0) t_ahead = claim();
+    // The barrier publishes task k+1 (broadcast at the end of task k-1 by
+    // rank 0's thread 0) and ends every thread's use of the buffer that the
+    // copies issued next land in (task k-1's).  With two buffers the copies
+    // of task k+1 stream in while task k computes; with one, the other CTA
+    // on the SM covers the copy of task k.
+    cluster_barrier_relaxed();
+    issue_loads(sh.task[(k + kTVBuffers - 1) & 3], (k + kTVBuffers - 1) % kTVBuffers);
 
-    const int bb = k & 1;
-    const unsigned parity = (unsigned)(k >> 1) & 1u;
+    const int bb = k % kTVBuffers;
     Tin* st = buf_t(bb);
     Tin* sd = buf_d(bb);
-    const TaskRows tr = task_rows(A, t);
-    const int pos = tr.pos, b = tr.b;
-    if (!A.aligned) {
-      const Tin *rt, *rd;
-      row_ptrs(pos, rt, rd);
-      for (int e = tid; e < len; e += kTVThreads) {
-        st[e] = rt[e];
-        sd[e] = rd[e];
+    int kind, idx;
+    decode_task(A, t, kind, idx);
+    unsigned parity = 0;
+    if (kind != kTaskS) {
+      parity = uses[bb] & 1u;
+      if (A.aligned) {
+        ++uses[bb];
+      } else {
+        const Tin *rt, *rd;
+        row_ptrs(idx, rt, rd);
+        for (int e = tid; e < len; e += kTVThreads) {
+          st[e] = rt[e];
+          sd[e] = rd[e];
+        }
+        __syncthreads();
       }
-      __syncthreads();
     }
 
-    if (tr.isA) {
+    if (kind == kTaskA) {
       // ---------------------------------------------------------- A-task
-      // pass 1: online max / sum-exp of both rows (log2 units), chunk by chunk
-      float mt = -INFINITY, ssum_t = 0.f, md = -INFINITY, ssum_d = 0.f;
+      const int pos = idx, b = pos / W;
+      // pass 0: row maxima of this slice (packed compares), chunk by chunk as
+      // the copies land; pass 1: sum of 2^(x - max) from shared memory.
+      float mt = -INFINITY, md = -INFINITY;
       for (int c = 0; c < kTVChunks; ++c) {
         const int e0 = c * chunk_elems;
         const int e1 = min(len, e0 + chunk_elems);
@@ -289,36 +364,73 @@ __global__ void __launch_bounds__(kTVThreads, 1) e2e_tv_kernel(const TVArgs A) {
         if (e1 <= e0) continue;
         const int nv = (e1 - e0) / VN;
         for (int vi = tid; vi < nv; vi += kTVThreads) {
-          const uint4 ut = *reinterpret_cast<const uint4*>(st + e0 + vi * VN);
-          const uint4 ud = *reinterpret_cast<const uint4*>(sd + e0 + vi * VN);
-          float ft[VN], fd[VN];
-          Vec<Tin>::unpack(ut, ft);
-          Vec<Tin>::unpack(ud, fd);
-#pragma unroll
-          for (int q = 0; q < VN; ++q) { ft[q] *= kLog2e; fd[q] *= kLog2e; }
-          online_update<VN>(mt, ssum_t, ft);
-          online_update<VN>(md, ssum_d, fd);
+          mt = fmaxf(mt, Vec<Tin>::vmax(*reinterpret_cast<const uint4*>(st + e0 + vi * VN)));
+          md = fmaxf(md, Vec<Tin>::vmax(*reinterpret_cast<const uint4*>(sd + e0 + vi * VN)));
         }
         for (int e = e0 + nv * VN + tid; e < e1; e += kTVThreads) {  // ragged tail
-          float xt = Elt<Tin>::to_f(st[e]) * kLog2e;
-          float xd = Elt<Tin>::to_f(sd[e]) * kLog2e;
-          online_update<1>(mt, ssum_t, &xt);
-          online_update<1>(md, ssum_d, &xd);
+          mt = fmaxf(mt, Elt<Tin>::to_f(st[e]));
+          md = fmaxf(md, Elt<Tin>::to_f(sd[e]));
         }
       }
-      block_lse2(mt, ssum_t, sh.wred);
-      block_lse2(md, ssum_d, sh.wred);
-      if (tid == 0) sh.cl_red1 = make_float4(mt, ssum_t, md, ssum_d);
-      cluster.sync();
-      mt = -INFINITY; ssum_t = 0.f; md = -INFINITY; ssum_d = 0.f;
-      for (int r = 0; r < A.CL; ++r) {
-        const float4 v = *cluster.map_shared_rank(&sh.cl_red1, r);
-        lse2_combine(mt, ssum_t, v.x, v.y);
-        lse2_combine(md, ssum_d, v.z, v.w);
+      mt *= kLog2e;
+      md *= kLog2e;
+      // Same element-to-thread mapping as pass 0, so each thread's maximum
+      // covers exactly the elements it sums.
+      float ssum_t = 0.f, ssum_d = 0.f;
+      if (mt != -INFINITY || md != -INFINITY) {
+        for (int c = 0; c < kTVChunks; ++c) {
+          const int e0 = c * chunk_elems;
+          const int e1 = min(len, e0 + chunk_elems);
+          if (e1 <= e0) continue;
+          const int nv = (e1 - e0) / VN;
+          for (int vi = tid; vi < nv; vi += kTVThreads) {
+            const uint4 ut = *reinterpret_cast<const uint4*>(st + e0 + vi * VN);
+            const uint4 ud = *reinterpret_cast<const uint4*>(sd + e0 + vi * VN);
+            float ft[VN], fd[VN];
+            Vec<Tin>::unpack(ut, ft);
+            Vec<Tin>::unpack(ud, fd);
+#pragma unroll
+            for (int q = 0; q < VN; ++q) {
+              ssum_t += exp2f(__fmaf_rn(ft[q], kLog2e, -mt));
+              ssum_d += exp2f(__fmaf_rn(fd[q], kLog2e, -md));
+            }
+          }
+          for (int e = e0 + nv * VN + tid; e < e1; e += kTVThreads) {
+            ssum_t += exp2f(__fmaf_rn(Elt<Tin>::to_f(st[e]), kLog2e, -mt));
+            ssum_d += exp2f(__fmaf_rn(Elt<Tin>::to_f(sd[e]), kLog2e, -md));
+          }
+        }
       }
-      const float lse2_t = mt + log2f(ssum_t);
-      const float lse2_d = md + log2f(ssum_d);
-      // pass 2: overlap and masked draft mass, from shared memory
+      // A -inf maximum means this thread saw no finite entry of that row: no
+      // mass (the NaNs formed above are dropped; the combine skips -inf).
+      if (mt == -INFINITY) ssum_t = 0.f;
+      if (md == -INFINITY) ssum_d = 0.f;
+      warp_lse2(mt, ssum_t);
+      warp_lse2(md, ssum_d);
+      if (lane == 0) sh.red_lse[warp] = make_float4(mt, ssum_t, md, ssum_d);
+      __syncthreads();
+      if (warp == 0) {
+        float4 v = lane < kTVWarps ? sh.red_lse[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        warp_lse2(v.x, v.y);
+        warp_lse2(v.z, v.w);
+        if (lane == 0) {
+          sh.cl_lse = v;
+          publish_for_cluster();
+        }
+      }
+      cluster_barrier_relaxed();
+      if (warp == 0) {
+        // lane r reads rank r's statistics: one DSMEM round trip
+        float4 v = lane < A.CL ? *cluster.map_shared_rank(&sh.cl_lse, lane)
+                               : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        warp_lse2(v.x, v.y);
+        warp_lse2(v.z, v.w);
+        if (lane == 0) sh.all_lse = v;
+      }
+      __syncthreads();
+      const float4 L = sh.all_lse;
+      const float lse2_t = L.x + log2f(L.y);
+      const float lse2_d = L.z + log2f(L.w);
       float pa = 0.f, ps = 0.f;
       {
         const int nv = len / VN;
@@ -345,85 +457,60 @@ __global__ void __launch_bounds__(kTVThreads, 1) e2e_tv_kernel(const TVArgs A) {
           ps += (ld < lt) ? ex : 0.f;
         }
       }
-      pa = block_sum(pa, sh.fred);
-      ps = block_sum(ps, sh.fred2);
-      if (tid == 0) sh.cl_red2 = make_float2(pa, ps);
-      cluster.sync();
-      if (rank == 0) {
-        float a_val = 0.f, s_val = 0.f;
-        for (int r = 0; r < A.CL; ++r) {
-          const float2 v = *cluster.map_shared_rank(&sh.cl_red2, r);
-          a_val += v.x;
-          s_val += v.y;
-        }
-        int last_all = 0;
-        if (tid == 0) {
-          const bool finite = (mt != -INFINITY) && (md != -INFINITY);
-          if (!tr.row_ok) set_status(SPECOPD_DEV_ROW_RANGE);
-          if (!finite) set_status(SPECOPD_DEV_ALL_NEG_INF);
-          if (!tr.row_ok || !finite) { a_val = __int_as_float(0x7fc00000); s_val = a_val; }
-          A.rec[pos] = make_float4(lse2_t, lse2_d, s_val, 0.f);
-          A.a_out[pos] = a_val;
-          __threadfence();
-          const unsigned old = atomicAdd(&A.cnt[b], 1u);
-          if (old == (unsigned)A.W - 1u) {
-            // This task completes branch b: prefix scan + gradient coefficients.
-            __threadfence();
-            const int base = b * A.W;
-            float P = 1.f;
-            double sumP = 0.0;
-            for (int i = 0; i < A.W; ++i) {
-              P *= __ldcg(&A.a_out[base + i]);
-              A.prefix[base + i] = P;
-              sumP += (double)P;
-            }
-            float S = 1.f;
-            for (int i = A.W - 1; i >= 0; --i) {
-              const float Pprev = (i == 0) ? 1.f : A.prefix[base + i - 1];
-              reinterpret_cast<float*>(&A.rec[base + i])[3] = -A.inv_norm * Pprev * S;
-              S = fmaf(__ldcg(&A.a_out[base + i]), S, 1.f);
-            }
-            A.bsum[b] = sumP;
-            __threadfence();
-            st_release_gpu(&A.ready[b], 1u);
-            const unsigned done = atomicAdd(&A.ctl[1], 1u);
-            if (done == (unsigned)A.nbranch - 1u) { __threadfence(); last_all = 1; }
-          }
-          sh.flag = last_all;
-        }
-        __syncthreads();
-        if (sh.flag) {
-          // Last branch: loss = 1 - sum_b bsum[b] / norm, fixed summation order.
-          double acc = 0.0;
-          for (int i = tid; i < A.nbranch; i += kTVThreads) acc += __ldcg(&A.bsum[i]);
-          acc = warp_sum_d(acc);
-          __syncthreads();
-          if ((tid & 31) == 0) sh.dred[tid >> 5] = acc;
-          __syncthreads();
-          if (tid == 0) {
-            double tot = 0.0;
-            for (int w = 0; w < kTVWarps; ++w) tot += sh.dred[w];
-            A.loss[0] = (float)(1.0 - tot / A.norm);
-            if (A.numer) A.numer[0] = tot;
-          }
+      pa = warp_sum(pa);
+      ps = warp_sum(ps);
+      if (lane == 0) sh.red_as[warp] = make_float2(pa, ps);
+      __syncthreads();
+      if (warp == 0) {
+        float2 v = lane < kTVWarps ? sh.red_as[lane] : make_float2(0.f, 0.f);
+        v.x = warp_sum(v.x);
+        v.y = warp_sum(v.y);
+        if (lane == 0) {
+          sh.cl_as = v;
+          publish_for_cluster();
         }
       }
-    } else {
+      cluster_barrier_relaxed();
+      if (rank == 0 && warp == 0) {
+        float2 v = lane < A.CL ? *cluster.map_shared_rank(&sh.cl_as, lane) : make_float2(0.f, 0.f);
+        v.x = warp_sum(v.x);
+        v.y = warp_sum(v.y);
+        if (lane == 0) {
+          const int trow = A.trow ? A.trow[pos] : pos;
+          const bool row_ok = (trow >= 0 && trow < A.rows_target);
+          const bool finite = (L.x != -INFINITY) && (L.z != -INFINITY);
+          if (!row_ok) set_status(SPECOPD_DEV_ROW_RANGE);
+          if (!finite) set_status(SPECOPD_DEV_ALL_NEG_INF);
+          if (!row_ok || !finite) v = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+          A.rec[pos] = make_float4(lse2_t, lse2_d, v.y, 0.f);
+          A.a_out[pos] = v.x;
+          // release: the two stores above are visible before the count
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&A.cnt[b]) : "memory");
+        }
+      }
+    } else if (kind == kTaskG) {
       // ---------------------------------------------------------- G-task
+      const int pos = idx, b = pos / W, i = pos % W;
       if (A.aligned) {
         for (int c = 0; c < kTVChunks; ++c)
           if (!mbar_wait(&sh.bar[bb][c], parity) && tid == 0) atomicExch(&A.ctl[2], 1u);
       }
-      if (tid == 0) {
-        const bool ok = wait_flag_geq(&A.ready[b], 1u);
-        if (!ok) atomicExch(&A.ctl[2], 1u);
-        sh.flag = ok ? 1 : 0;
+      const bool ok = stage_branch(b);
+      if (ok && tid == 0) {
+        // g = -(1/norm) P_{i-1} S_i  (no division by any overlap)
+        float P = 1.f;
+        for (int j = 0; j < i; ++j) P *= sh.sa[j];
+        float S = 1.f;
+        for (int j = W - 1; j > i; --j) S = fmaf(sh.sa[j], S, 1.f);
+        sh.g = -A.inv_norm * P * S;
       }
       __syncthreads();
-      const int ok = sh.flag;
+      // G(b, 1) publishes the branch's prefix products before its gradient
+      // stores, so its fence does not wait for them.
+      if (ok && i == 0 && rank == 0) scan_branch(b);
       if (ok && len > 0) {
         const float4 r = __ldcg(&A.rec[pos]);
-        const float lse2_t = r.x, lse2_d = r.y, s_val = r.z, g = r.w;
+        const float lse2_t = r.x, lse2_d = r.y, s_val = r.z, g = sh.g;
         Tg* gout = reinterpret_cast<Tg*>(A.grad) + (long long)pos * V + v0;
         if (A.aligned) {
           const int nv = len / VN;
@@ -466,18 +553,25 @@ __global__ void __launch_bounds__(kTVThreads, 1) e2e_tv_kernel(const TVArgs A) {
           }
         }
       }
+    } else {
+      // ---------------------------------------------------------- S-task
+      if (rank == 0 && stage_branch(idx)) scan_branch(idx);
+    }
+    if (rank == 0 && tid == 0) {
+      broadcast((k + 2) & 3, t_ahead);
+      publish_for_cluster();
     }
   }
   // Rank 0 may still be reading a peer's shared memory (DSMEM) from the last
   // task; no CTA of the cluster may exit before every peer is done with it.
-  cluster.sync();
+  cluster_barrier_relaxed();
 }
 
 // ------------------------------------------------------------------ host
 namespace {
 
 struct TVLayout {
-  size_t rec, bsum, cnt, ready, ctl, total, zero_begin, zero_bytes;
+  size_t rec, bsum, cnt, ctl, total, zero_begin, zero_bytes;
 };
 
 TVLayout tv_layout(const TVProblem& p) {
@@ -487,7 +581,6 @@ TVLayout tv_layout(const TVProblem& p) {
   L.rec = off;   off = up(off + sizeof(float4) * (size_t)p.N);
   L.bsum = off;  off = up(off + sizeof(double) * (size_t)p.nbranch);
   L.cnt = off;   off += sizeof(unsigned) * (size_t)p.nbranch;
-  L.ready = off; off += sizeof(unsigned) * (size_t)p.nbranch;
   L.ctl = off;   off = up(off + 4 * sizeof(unsigned));
   L.zero_begin = L.cnt;
   L.zero_bytes = off - L.cnt;
@@ -521,16 +614,17 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
                           void* grad, void* ws, size_t ws_bytes, cudaStream_t stream) {
   const TVLayout L = tv_layout(p);
   if (ws_bytes < L.total) return cudaErrorInvalidValue;
+  if (p.W > kTVMaxW) return cudaErrorInvalidConfiguration;
   const int es = elt_size(p.logit_dtype);
   const int gs = elt_size(p.grad_dtype);
-  // Cluster size: smallest CL whose per-CTA slice of both rows fits the budget.
-  int CL = (int)((4ll * p.V * es + kTVSmemBudget - 1) / kTVSmemBudget);
+  // Cluster size: smallest CL whose per-CTA slices of two tasks fit the budget.
+  int CL = (int)((2ll * kTVBuffers * p.V * es + kTVSmemBudget - 1) / kTVSmemBudget);
   if (CL < 1) CL = 1;
   int Lc = (p.V + CL - 1) / CL;
   Lc = (Lc + 15) / 16 * 16;
   CL = (p.V + Lc - 1) / Lc;
   if (CL > 16) return cudaErrorInvalidConfiguration;
-  const size_t smem = ((sizeof(TVShared) + 127) / 128) * 128 + 4ull * Lc * es;
+  const size_t smem = ((sizeof(TVShared) + 127) / 128) * 128 + 2ull * kTVBuffers * Lc * es;
 
   TVArgs A;
   A.nbranch = p.nbranch; A.W = p.W; A.V = p.V; A.N = p.N; A.rows_target = p.rows_target;
@@ -547,7 +641,6 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
   A.rec = reinterpret_cast<float4*>(w + L.rec);
   A.bsum = reinterpret_cast<double*>(w + L.bsum);
   A.cnt = reinterpret_cast<unsigned*>(w + L.cnt);
-  A.ready = reinterpret_cast<unsigned*>(w + L.ready);
   A.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
 
   void* fn = pick_kernel(p.logit_dtype, p.grad_dtype);
@@ -593,7 +686,7 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
       g_occ_cache[key] = nclusters;
     }
   }
-  A.total_tasks = p.N * (A.compute_grad ? 2 : 1);
+  A.total_tasks = p.N + (A.compute_grad ? p.N : p.nbranch);
   if (nclusters > A.total_tasks) nclusters = A.total_tasks;
   A.lag = (nclusters + p.W - 1) / p.W + 1;
   cfg.gridDim = dim3(CL * nclusters);

@@ -381,6 +381,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int b = j & 1;
       if (!warp_wait_or_abort(&hdr->s_full[b], (j >> 1) & 1, hdr)) break;
       tc_fence_after();
+      __syncwarp();  // tcgen05.ld/st are warp-collective (.sync.aligned)
 #pragma unroll
       for (int q = 0; q < kBN / 32; ++q) tmem_ld32(tS[b] + lane_off + q * 32, sv + q * 32);
       tmem_wait_ld();
@@ -418,6 +419,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           // O holds PV of tiles < j; PV of tile j-1 must be complete.
           if (!warp_wait_or_abort(&hdr->o_done, (j - 1) & 1, hdr)) break;
           tc_fence_after();
+          __syncwarp();
 #pragma unroll
           for (int q = 0; q < D / 32; ++q) {
             uint32_t ov[32];
@@ -441,6 +443,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         pk[e] = pack_bf16x2(p0, p1);
       }
       l += rs;
+      __syncwarp();
       tmem_st32(tS[b] + lane_off, pk);
       tmem_st32(tS[b] + lane_off + 32, pk + 32);
       tmem_wait_st();
@@ -451,6 +454,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float o[D];
     const bool ok = warp_wait_or_abort(&hdr->o_final, 0, hdr) && !hdr->abort;
     tc_fence_after();
+    __syncwarp();
 #pragma unroll
     for (int q = 0; q < D / 32; ++q) {
       uint32_t ov[32];
