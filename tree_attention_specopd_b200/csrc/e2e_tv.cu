@@ -219,6 +219,8 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
   auto buf_t = [&](int bb) { return buf0 + (size_t)bb * 2 * A.Lc; };
   auto buf_d = [&](int bb) { return buf0 + (size_t)bb * 2 * A.Lc + A.Lc; };
 
+  const uint64_t pol_keep = l2_policy_evict_last();
+  const uint64_t pol_drop = l2_policy_evict_first();
   // Start the bulk copies of task t's rows into buffer bb (aligned path; A and
   // G tasks only -- S tasks touch no rows).
   auto issue_loads = [&](int t, int bb) {
@@ -237,8 +239,11 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
       const unsigned bytes = e1 > e0 ? (unsigned)((e1 - e0) * sizeof(Tin)) : 0u;
       mbar_arrive_expect_tx(&sh.bar[bb][c], 2u * bytes);
       if (bytes) {
-        bulk_g2s(st + e0, rt + e0, bytes, &sh.bar[bb][c]);
-        bulk_g2s(sd + e0, rd + e0, bytes, &sh.bar[bb][c]);
+        // A-task rows are read again by the branch's G-tasks shortly after:
+        // keep them in L2 (evict_last); a G-task is their last use.
+        const uint64_t pol = kind == kTaskA ? pol_keep : pol_drop;
+        bulk_g2s_hint(st + e0, rt + e0, bytes, &sh.bar[bb][c], pol);
+        bulk_g2s_hint(sd + e0, rd + e0, bytes, &sh.bar[bb][c], pol);
       }
     }
   };
@@ -247,8 +252,8 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
   unsigned uses[kTVBuffers] = {};
 
   auto claim = [&]() -> int {
-    int t = A.total_tasks;
-    if (*((volatile unsigned*)&A.ctl[2]) == 0u) t = (int)atomicAdd(&A.ctl[0], 1u);
+    const int t = (int)atomicAdd(&A.ctl[0], 1u);
+    if (__ldcg(&A.ctl[2]) != 0u) return A.total_tasks;  // a wait ran out: stop
     return t > A.total_tasks ? A.total_tasks : t;
   };
   auto broadcast = [&](int slot, int t) {
@@ -319,9 +324,7 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
   for (int k = 0;; ++k) {
     const int t = sh.task[k & 3];
     if (t >= A.total_tasks) break;
-    // Claim task k+2 now; its id is broadcast at the end of this task.
-    int t_ahead = A.total_tasks;
-    if (rank == 0 && tid == 0) t_ahead = claim();
+
     // The barrier publishes task k+1 (broadcast at the end of task k-1 by
     // rank 0's thread 0) and ends every thread's use of the buffer that the
     // copies issued next land in (task k-1's).  With two buffers the copies
@@ -329,6 +332,10 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
     // on the SM covers the copy of task k.
     cluster_barrier_relaxed();
     issue_loads(sh.task[(k + kTVBuffers - 1) & 3], (k + kTVBuffers - 1) % kTVBuffers);
+    // Claim task k+2 (warp 1, so thread 0's copies are not delayed); the id
+    // is only needed when it is broadcast at the end of this task.
+    int t_ahead = A.total_tasks;
+    if (rank == 0 && tid == 32) t_ahead = claim();
 
     const int bb = k % kTVBuffers;
     Tin* st = buf_t(bb);
@@ -354,6 +361,11 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
     if (kind == kTaskA) {
       // ---------------------------------------------------------- A-task
       const int pos = idx, b = pos / W;
+      bool task_row_ok = true;
+      if (rank == 0 && tid == 0 && A.trow) {
+        const int trow = A.trow[pos];  // read early; used when publishing
+        task_row_ok = (trow >= 0 && trow < A.rows_target);
+      }
       // pass 0: row maxima of this slice (packed compares), chunk by chunk as
       // the copies land; pass 1: sum of 2^(x - max) from shared memory.
       float mt = -INFINITY, md = -INFINITY;
@@ -389,11 +401,22 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
             float ft[VN], fd[VN];
             Vec<Tin>::unpack(ut, ft);
             Vec<Tin>::unpack(ud, fd);
+            // independent partial sums: no serial FADD chain across the vector
+            float at[VN], ad[VN];
 #pragma unroll
             for (int q = 0; q < VN; ++q) {
-              ssum_t += exp2f(__fmaf_rn(ft[q], kLog2e, -mt));
-              ssum_d += exp2f(__fmaf_rn(fd[q], kLog2e, -md));
+              at[q] = exp2f(__fmaf_rn(ft[q], kLog2e, -mt));
+              ad[q] = exp2f(__fmaf_rn(fd[q], kLog2e, -md));
             }
+#pragma unroll
+            for (int w = VN / 2; w > 0; w >>= 1)
+#pragma unroll
+              for (int q = 0; q < w; ++q) {
+                at[q] += at[q + w];
+                ad[q] += ad[q + w];
+              }
+            ssum_t += at[0];
+            ssum_d += ad[0];
           }
           for (int e = e0 + nv * VN + tid; e < e1; e += kTVThreads) {
             ssum_t += exp2f(__fmaf_rn(Elt<Tin>::to_f(st[e]), kLog2e, -mt));
@@ -440,14 +463,23 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
           float ft[VN], fd[VN];
           Vec<Tin>::unpack(ut, ft);
           Vec<Tin>::unpack(ud, fd);
+          float ea[VN], es[VN];
 #pragma unroll
           for (int q = 0; q < VN; ++q) {
             const float lt = __fmaf_rn(ft[q], kLog2e, -lse2_t);
             const float ld = __fmaf_rn(fd[q], kLog2e, -lse2_d);
-            const float e = exp2f(fminf(lt, ld));
-            pa += e;
-            ps += (ld < lt) ? e : 0.f;
+            ea[q] = exp2f(fminf(lt, ld));
+            es[q] = (ld < lt) ? ea[q] : 0.f;
           }
+#pragma unroll
+          for (int w = VN / 2; w > 0; w >>= 1)
+#pragma unroll
+            for (int q = 0; q < w; ++q) {
+              ea[q] += ea[q + w];
+              es[q] += es[q + w];
+            }
+          pa += ea[0];
+          ps += es[0];
         }
         for (int e = nv * VN + tid; e < len; e += kTVThreads) {
           const float lt = __fmaf_rn(Elt<Tin>::to_f(st[e]), kLog2e, -lse2_t);
@@ -476,8 +508,7 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
         v.x = warp_sum(v.x);
         v.y = warp_sum(v.y);
         if (lane == 0) {
-          const int trow = A.trow ? A.trow[pos] : pos;
-          const bool row_ok = (trow >= 0 && trow < A.rows_target);
+          const bool row_ok = task_row_ok;
           const bool finite = (L.x != -INFINITY) && (L.z != -INFINITY);
           if (!row_ok) set_status(SPECOPD_DEV_ROW_RANGE);
           if (!finite) set_status(SPECOPD_DEV_ALL_NEG_INF);
@@ -557,7 +588,7 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
       // ---------------------------------------------------------- S-task
       if (rank == 0 && stage_branch(idx)) scan_branch(idx);
     }
-    if (rank == 0 && tid == 0) {
+    if (rank == 0 && tid == 32) {
       broadcast((k + 2) & 3, t_ahead);
       publish_for_cluster();
     }
@@ -688,7 +719,9 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
   }
   A.total_tasks = p.N + (A.compute_grad ? p.N : p.nbranch);
   if (nclusters > A.total_tasks) nclusters = A.total_tasks;
-  A.lag = (nclusters + p.W - 1) / p.W + 1;
+  // G-tasks of a branch start ~2 rounds of the whole grid after its A-tasks,
+  // so they rarely wait, while its rows are still resident in L2.
+  A.lag = (2 * nclusters + p.W - 1) / p.W + 1;
   cfg.gridDim = dim3(CL * nclusters);
   void* args[] = {&A};
   return cudaLaunchKernelExC(&cfg, fn, args);

@@ -42,7 +42,7 @@
 namespace specopd {
 namespace sm100 {
 
-constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2..5: softmax
+constexpr int kThreads = 320;  // warp 0: TMA, warp 1: MMA, warps 2..9: softmax
 constexpr int kBN = 128;       // keys per tile
 constexpr int kStages = 2;     // K and V ring depth
 constexpr int kTmemCols = 512;
@@ -71,6 +71,8 @@ struct Hdr {
   uint64_t o_done;   // one phase per P.V tile (used by the lazy rescale)
   uint64_t o_final;  // single phase: every MMA of the unit has completed
   uint32_t tmem_base;
+  float red_max[2][2][128];  // [tile parity][column half][row] partial maxima
+  float red_sum[2][128];     // [column half][row] partial sums
   int kmax;
   int last;
   int abort;
@@ -179,7 +181,10 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Bounded wait; once any wait of the CTA has run out (hdr->abort), later
+// waits return false at once, so an aborting CTA finishes quickly.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, Hdr* hdr) {
+  if (*reinterpret_cast<volatile int*>(&hdr->abort)) return false;
   if (mbar_wait(bar, parity)) return true;
   hdr->abort = 1;
   return false;
@@ -188,7 +193,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, unsigned parity, Hd
 // Same, for the softmax warps: the result is uniform over the warp, because
 // the tcgen05.ld/st that follow are warp-collective (.sync.aligned).
 __device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, unsigned parity, Hdr* hdr) {
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity));
+  const bool live = !*reinterpret_cast<volatile int*>(&hdr->abort);
+  const bool ok = __all_sync(0xffffffffu, live && mbar_wait(bar, parity));
   if (!ok) hdr->abort = 1;
   return ok;
 }
@@ -255,7 +261,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&hdr->s_full[i], 1);
-      mbar_init(&hdr->p_full[i], 128);
+      mbar_init(&hdr->p_full[i], 256);
     }
     mbar_init(&hdr->o_done, 1);
     mbar_init(&hdr->o_final, 1);
@@ -358,7 +364,13 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else {
     // ================================================================ softmax / epilogue
+    // Eight warps: two per TMEM lane quadrant (warp & 3); the warp's half h2
+    // owns columns [64*h2, 64*h2 + 64) of its 32 rows' S tiles and columns
+    // [DH*h2, DH*h2 + DH) of O.  The two halves of a row exchange their
+    // partial maxima through shared memory once per tile.
+    constexpr int DH = D / 2;
     const int q4 = warp & 3;             // TMEM lane quadrant of this warp
+    const int h2 = (warp - 2) >> 2;      // column half
     const int mrow = q4 * 32 + lane;     // query row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const int G = P.G;
@@ -375,17 +387,27 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     const bool live = in_tile && !bad;
     const float sl2 = P.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    uint32_t sv[kBN];
+    const int c0 = 64 * h2;              // first S column of this half
+    float m = -INFINITY, l = 0.f;        // running max (log2 units) and this half's sum
+    uint32_t sv[64];
+    // After a wait runs out the warp keeps stepping through the loop with its
+    // TMEM work skipped (dead), so the named barriers shared by the eight
+    // softmax warps still match.
+    bool dead = false;
     for (int j = 0; j < nk; ++j) {
       const int b = j & 1;
-      if (!warp_wait_or_abort(&hdr->s_full[b], (j >> 1) & 1, hdr)) break;
-      tc_fence_after();
-      __syncwarp();  // tcgen05.ld/st are warp-collective (.sync.aligned)
+      if (!dead) dead = !warp_wait_or_abort(&hdr->s_full[b], (j >> 1) & 1, hdr);
+      if (!dead) {
+        tc_fence_after();
+        __syncwarp();  // tcgen05.ld/st are warp-collective (.sync.aligned)
+        tmem_ld32(tS[b] + lane_off + c0, sv);
+        tmem_ld32(tS[b] + lane_off + c0 + 32, sv + 32);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) tmem_ld32(tS[b] + lane_off + q * 32, sv + q * 32);
-      tmem_wait_ld();
-      // visible columns: lo <= col <= hi
+        for (int e = 0; e < 64; ++e) sv[e] = 0u;
+      }
+      // visible columns of the tile: lo <= col <= hi
       int lo, hi;
       if (j < nt) {
         lo = 0;
@@ -396,13 +418,25 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         hi = r - node0;
       }
       if (!live) hi = -1;
-      float mx = -INFINITY;
+      // raw-score maximum (the scale is positive, so it commutes with max)
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (__all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 63)) {
+        // every column of this half is visible to every row of the warp
 #pragma unroll
-      for (int col = 0; col < kBN; ++col) {
-        const float x = (col >= lo && col <= hi) ? __uint_as_float(sv[col]) * sl2 : -INFINITY;
-        sv[col] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int e = 0; e < 64; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(sv[e]));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const int col = c0 + e;
+          const float x = (col >= lo && col <= hi) ? __uint_as_float(sv[e]) : -INFINITY;
+          sv[e] = __float_as_uint(x);
+          mx4[e & 3] = fmaxf(mx4[e & 3], x);
+        }
       }
+      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      hdr->red_max[b][h2][mrow] = mx;
+      named_bar_sync(1, 256);
+      mx = fmaxf(mx, hdr->red_max[b][h2 ^ 1][mrow]) * sl2;
       const float m_new = fmaxf(m, mx);
       // Lazy rescale: keep the stale max unless it grew by more than 2^8.
       const bool need = (m != -INFINITY) && (m_new > m + kRescaleThreshold);
@@ -415,61 +449,66 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           l *= f;
           m = m_new;
         }
-        if (j > 0) {
+        if (j > 0 && !dead) dead = !warp_wait_or_abort(&hdr->o_done, (j - 1) & 1, hdr);
+        if (j > 0 && !dead) {
           // O holds PV of tiles < j; PV of tile j-1 must be complete.
-          if (!warp_wait_or_abort(&hdr->o_done, (j - 1) & 1, hdr)) break;
           tc_fence_after();
           __syncwarp();
 #pragma unroll
-          for (int q = 0; q < D / 32; ++q) {
+          for (int q = 0; q < DH / 32; ++q) {
             uint32_t ov[32];
-            tmem_ld32(tO + lane_off + q * 32, ov);
+            tmem_ld32(tO + lane_off + DH * h2 + q * 32, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-            tmem_st32(tO + lane_off + q * 32, ov);
+            tmem_st32(tO + lane_off + DH * h2 + q * 32, ov);
           }
         }
       }
-      float rs = 0.f;
-      uint32_t pk[kBN / 2];
+      // p = 2^(s*scale*log2e - m); masked entries are -inf -> 0
+      const float nm = (m == -INFINITY) ? 0.f : -m;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
 #pragma unroll
-      for (int e = 0; e < kBN / 2; ++e) {
-        const float x0 = __uint_as_float(sv[2 * e]);
-        const float x1 = __uint_as_float(sv[2 * e + 1]);
-        const float p0 = (m == -INFINITY) ? 0.f : exp2f(x0 - m);
-        const float p1 = (m == -INFINITY) ? 0.f : exp2f(x1 - m);
-        rs += p0 + p1;
+      for (int e = 0; e < 32; ++e) {
+        const float p0 = exp2f(__fmaf_rn(__uint_as_float(sv[2 * e]), sl2, nm));
+        const float p1 = exp2f(__fmaf_rn(__uint_as_float(sv[2 * e + 1]), sl2, nm));
+        rs4[e & 3] += p0 + p1;
         pk[e] = pack_bf16x2(p0, p1);
       }
-      l += rs;
-      __syncwarp();
-      tmem_st32(tS[b] + lane_off, pk);
-      tmem_st32(tS[b] + lane_off + 32, pk + 32);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&hdr->p_full[b]);
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      if (!dead) {
+        __syncwarp();
+        tmem_st32(tS[b] + lane_off + 32 * h2, pk);  // P of keys [c0, c0+64) as bf16 pairs
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&hdr->p_full[b]);
+      }
     }
     // ---- epilogue
-    float o[D];
+    float o[DH];
     const bool ok = warp_wait_or_abort(&hdr->o_final, 0, hdr) && !hdr->abort;
     tc_fence_after();
     __syncwarp();
 #pragma unroll
-    for (int q = 0; q < D / 32; ++q) {
+    for (int q = 0; q < DH / 32; ++q) {
       uint32_t ov[32];
-      tmem_ld32(tO + lane_off + q * 32, ov);
+      tmem_ld32(tO + lane_off + DH * h2 + q * 32, ov);
       tmem_wait_ld();
 #pragma unroll
       for (int e = 0; e < 32; ++e) o[q * 32 + e] = __uint_as_float(ov[e]);
     }
+    // row sum = both halves' partial sums (same reference max)
+    hdr->red_sum[h2][mrow] = l;
+    named_bar_sync(1, 256);
+    l += hdr->red_sum[h2 ^ 1][mrow];
     const int hq = h * G + g;
     const float qnan = __int_as_float(0x7fc00000);
     auto write_row = [&](const float* acc, float mm, float ll) {
-      __nv_bfloat16* dst = P.out + ((size_t)r * P.Hq + hq) * D;
+      __nv_bfloat16* dst = P.out + ((size_t)r * P.Hq + hq) * D + DH * h2;
       const float inv = (bad || !ok) ? qnan : 1.f / ll;
 #pragma unroll
-      for (int e = 0; e < D; e += 8) {
+      for (int e = 0; e < DH; e += 8) {
         uint4 v;
         v.x = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
         v.y = pack_bf16x2(acc[e + 2] * inv, acc[e + 3] * inv);
@@ -477,8 +516,10 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         v.w = pack_bf16x2(acc[e + 6] * inv, acc[e + 7] * inv);
         *reinterpret_cast<uint4*>(dst + e) = v;
       }
-      if (P.lse) P.lse[(size_t)r * P.Hq + hq] = (bad || !ok) ? qnan : (mm + log2f(ll)) * 0.6931471805599453f;
-      if (bad && g == 0) set_status(SPECOPD_DEV_ANCHOR_RANGE);
+      if (h2 == 0) {
+        if (P.lse) P.lse[(size_t)r * P.Hq + hq] = (bad || !ok) ? qnan : (mm + log2f(ll)) * 0.6931471805599453f;
+        if (bad && g == 0) set_status(SPECOPD_DEV_ANCHOR_RANGE);
+      }
     };
     if (nact == 1) {
       if (in_tile) write_row(o, m, l);
@@ -488,18 +529,20 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const size_t slot_floats = (size_t)128 * D + 256;
       float* mine = P.part + (slot + c) * slot_floats;
 #pragma unroll
-      for (int e = 0; e < D; e += 4)
-        __stcg(reinterpret_cast<float4*>(mine + (size_t)mrow * D + e),
+      for (int e = 0; e < DH; e += 4)
+        __stcg(reinterpret_cast<float4*>(mine + (size_t)mrow * D + DH * h2 + e),
                make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
-      mine[128 * D + mrow] = m;
-      mine[128 * D + 128 + mrow] = l;
+      if (h2 == 0) {
+        mine[128 * D + mrow] = m;
+        mine[128 * D + 128 + mrow] = l;
+      }
       __threadfence();
-      named_bar_sync(1, 128);
-      if (mrow == 0) {
+      named_bar_sync(1, 256);
+      if (mrow == 0 && h2 == 0) {
         const unsigned old = atomicAdd(&P.cnt[tile * P.Hkv + h], 1u);
         hdr->last = (old == (unsigned)nact - 1u) ? 1 : 0;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, 256);
       if (hdr->last) {
         __threadfence();
         float mm = -INFINITY;
@@ -507,15 +550,15 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           mm = fmaxf(mm, __ldcg(P.part + (slot + cc) * slot_floats + 128 * D + mrow));
         float ll = 0.f;
 #pragma unroll
-        for (int e = 0; e < D; ++e) o[e] = 0.f;
+        for (int e = 0; e < DH; ++e) o[e] = 0.f;
         for (int cc = 0; cc < nact; ++cc) {
           const float* pc = P.part + (slot + cc) * slot_floats;
           const float mc = __ldcg(pc + 128 * D + mrow);
           const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - mm);
           ll += wgt * __ldcg(pc + 128 * D + 128 + mrow);
 #pragma unroll
-          for (int e = 0; e < D; e += 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(pc + (size_t)mrow * D + e));
+          for (int e = 0; e < DH; e += 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(pc + (size_t)mrow * D + DH * h2 + e));
             o[e] += wgt * v.x;
             o[e + 1] += wgt * v.y;
             o[e + 2] += wgt * v.z;
