@@ -183,7 +183,7 @@ class Problem:
             ev[2].record()
 
 
-KERNELS_PER_STEP = 5  # tree_build, rope(q), rope(k), tree_attn, e2e_tv
+KERNELS_PER_STEP = 4  # tree_build, rope(branch q and k), tree_attn, e2e_tv
 
 
 def run_gpu(args):

@@ -224,9 +224,8 @@ specopd_status specopd_tree_attn(const specopd_attn_desc* d, const void* q_br, c
   rope_theta(p.D, d->rope_base, theta);
   // Branch q/k rotated once at their semantic positions (sem_pos of the
   // branch nodes); every key tile of a query tile reuses the rotated copy.
-  cudaError_t e = launch_rope(p.dtype, q_br, q_rot, sem_pos + p.T_tot, p.R, p.Hq, p.D, theta, st);
-  if (e == cudaSuccess)
-    e = launch_rope(p.dtype, k_br, k_rot, sem_pos + p.T_tot, p.R, p.Hkv, p.D, theta, st);
+  cudaError_t e = launch_rope2(p.dtype, q_br, q_rot, p.Hq, k_br, k_rot, p.Hkv, sem_pos + p.T_tot,
+                               p.R, p.D, theta, st);
   if (e != cudaSuccess) return cuda_status(e);
   if (p.dtype == SPECOPD_F32) {
     e = launch_attn_simt_f32(p, (const float*)q_rot, (const float*)k_rot, (const float*)v_br,

@@ -29,6 +29,10 @@ cudaError_t launch_tree_build(const CuTrunk& cu, const int32_t* anchors, int B, 
 // theta: host array of D/2 frequencies base^(-2k/D) in double precision.
 cudaError_t launch_rope(specopd_dtype dt, const void* x, void* y, const int32_t* pos, int n, int H,
                         int D, const double* theta_host, cudaStream_t st);
+// Two tensors (H0 and H1 heads) rotated at the same positions in one launch.
+cudaError_t launch_rope2(specopd_dtype dt, const void* x0, void* y0, int H0, const void* x1,
+                         void* y1, int H1, const int32_t* pos, int n, int D,
+                         const double* theta_host, cudaStream_t st);
 
 // ---- tree attention, SIMT (fp32 workloads)
 struct AttnProblem {
