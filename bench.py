@@ -191,6 +191,7 @@ def run_gpu(args):
     import torch.distributed as dist
 
     from tree_attention_specopd_b200 import api
+    from tree_attention_specopd_b200 import dist as sdist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -202,17 +203,21 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     api.load()
     pb = Problem(torch, api, dev, seed_offset=rank)
+    # Distributed normalisation: every rank's gradient and loss divide by the
+    # GLOBAL position count (gathered once), and the prefix-product sums are
+    # all-reduced after each step.
+    n_global = sdist.global_count(pb.N, device=dev)
     if world > 1:
-        # Eq. 18: the gradient and loss divide by the GLOBAL position count.
         pb.tdesc = api.tv_desc(pb.acfg.S * pb.acfg.B, pb.acfg.W, pb.V, pb.rows_t, "bf16", "f32",
-                               True, norm_count=pb.N * world)
+                               True, norm_count=n_global)
     numer_all = torch.zeros(1, dtype=torch.float64, device=dev)
+    loss_all = torch.zeros(1, dtype=torch.float64, device=dev)
 
     def full_step(ev=None):
         pb.step(ev)
         if world > 1:
             numer_all.copy_(pb.numer)
-            dist.all_reduce(numer_all)
+            loss_all.copy_(sdist.global_loss(numer_all, n_global))
 
     for _ in range(args.warmup):
         full_step()
