@@ -265,8 +265,8 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* desc,
  * SPECOPD_E2E_TV_STATIC_SCRATCH_BYTES in the library's device image, held by
  * every GPU that loads the library until the process exits.
  *   - Size limit: returns SPECOPD_ERR_WORKSPACE, launching nothing, when
- *     specopd_e2e_tv_workspace_size(desc) exceeds the array (1 MiB holds
- *     about 60,000 positions).
+ *     specopd_e2e_tv_workspace_size(desc) exceeds the array (8 MiB: about
+ *     30,000 positions at a 151,936-token bf16 vocabulary).
  *   - The first call on each device resolves the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - All calls on a device share the array, which keeps the last call's
@@ -274,7 +274,7 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* desc,
  *     overlap on the GPU -- other streams, other host threads -- race on it:
  *     serialise them.
  */
-#define SPECOPD_E2E_TV_STATIC_SCRATCH_BYTES (1u << 20)
+#define SPECOPD_E2E_TV_STATIC_SCRATCH_BYTES (8u << 20)
 
 specopd_status specopd_e2e_tv_noalloc(const specopd_tv_desc* desc,
                                       const void* z_target,

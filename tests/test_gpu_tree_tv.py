@@ -229,6 +229,7 @@ def test_tv_8b_bf16_through_score_rows(lib):
     (1001, 3, 5, "f32", "f32"),    # V not a multiple of the vector width (unaligned path)
     (1003, 2, 3, "bf16", "bf16"),  # odd row stride in bf16, bf16 grads
     (4096, 1, 7, "bf16", "f32"),   # W = 1
+    (1000, 3, 4, "f32", "bf16"),   # fp32 logits, bf16 gradient (aligned path)
     (111_104, 4, 2, "bf16", "f32"),  # cluster of 3 CTAs, ragged last slice, aligned path
 ])
 def test_tv_shapes(lib, V, W, nb, dtype, gdt):

@@ -72,8 +72,8 @@ def test_noalloc_matches_workspace_entry_point(nb, W, V, dtype, gather):
 
 
 def test_noalloc_rejects_sizes_beyond_the_array():
-    # 200,000 positions need more scratch than the fixed array holds.
-    desc = api.tv_desc(50_000, 4, 16, 200_000, "f32", "f32", True)
+    # 800,000 positions need more scratch than the fixed array holds.
+    desc = api.tv_desc(200_000, 4, 16, 800_000, "f32", "f32", True)
     assert api.specopd_e2e_tv_workspace_size(desc) > api.E2E_TV_STATIC_SCRATCH_BYTES
     dummy = torch.empty(1, device="cuda")
     with pytest.raises(api.SpecopdError) as ei:

@@ -226,13 +226,13 @@ def specopd_e2e_tv(desc, z_target, target_row, z_draft, a=None, prefix=None, los
     return {"a": a, "prefix": prefix, "loss": loss, "numer": numer, "grad": grad}
 
 
-E2E_TV_STATIC_SCRATCH_BYTES = 1 << 20
+E2E_TV_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 def specopd_e2e_tv_noalloc(desc, z_target, target_row, z_draft, a, prefix, loss, numer=None,
                            grad=None, stream=None):
     """E2E-TV without a workspace argument, for callers that cannot allocate
-    device memory (the library's fixed 1 MiB scratch array is used instead).
+    device memory (the library's fixed 8 MiB scratch array is used instead).
     All outputs are caller-provided; calls that overlap on the GPU race on the
     shared scratch and must be serialised."""
     _check(load().specopd_e2e_tv_noalloc(ctypes.byref(desc), _ptr(z_target), _ptr(target_row),

@@ -113,9 +113,8 @@ specopd_status tv_problem(const specopd_tv_desc* d, TVProblem& p) {
   p.logit_dtype = d->logit_dtype; p.grad_dtype = d->grad_dtype;
   p.compute_grad = d->compute_grad ? 1 : 0;
   p.norm_count = d->norm_count > 0 ? (double)d->norm_count : (double)N;
-  // Cluster size needed to hold both rows in shared memory (<= 16 CTAs).
-  const long long CL = (2ll * kTVBuffers * d->V * (long long)elt(d->logit_dtype) + kTVSmemBudget - 1) / kTVSmemBudget;
-  if (CL > 16) return SPECOPD_ERR_UNSUPPORTED;
+  // Slices per row (each CTA holds one slice of both rows in shared memory).
+  if (tv_slice_count(p) > kTVMaxSlices || d->W > kTVMaxW) return SPECOPD_ERR_UNSUPPORTED;
   return SPECOPD_OK;
 }
 

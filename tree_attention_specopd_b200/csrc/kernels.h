@@ -60,6 +60,7 @@ struct TVProblem {
   double norm_count;
 };
 size_t tv_workspace(const TVProblem& p);
+int tv_slice_count(const TVProblem& p);
 cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_t* target_row,
                           const void* z_draft, float* a, float* prefix, float* loss, double* numer,
                           void* grad, void* ws, size_t ws_bytes, cudaStream_t st);
