@@ -76,10 +76,10 @@ __device__ __forceinline__ unsigned atom_add_acqrel_gpu(unsigned* p, unsigned v)
 __device__ __forceinline__ bool wait_flag_geq(const unsigned* flag, unsigned want) {
   if (ld_acquire_gpu(flag) >= want) return true;
   const unsigned long long t0 = globaltimer_ns();
-  unsigned ns = 32;
+  // Short, fixed pause: the waits here last microseconds, and a growing
+  // back-off would overshoot the moment the flag flips.
   while (true) {
-    __nanosleep(ns);
-    if (ns < 1024) ns <<= 1;
+    __nanosleep(64);
     if (ld_acquire_gpu(flag) >= want) return true;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       set_status(SPECOPD_DEV_TIMEOUT);
@@ -165,6 +165,15 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+
+// 2^x with the hardware approximation (ex2.approx.ftz.f32: one MUFU op,
+// relative error about 2^-22; results below 2^-126 flush to zero, which a
+// softmax term that small never affects at fp32 precision).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ---------------------------------------------------------------- warp utils

@@ -21,7 +21,7 @@
 // exactly that.
 //  * Task = (position n, vocabulary slice c), NS slices per row.  A CTA
 //    (128 threads) holds one task: both rows' slice arrive by 1-D bulk copy
-//    (TMA) into its shared memory and stay there for all three passes.  Four
+//    (TMA) into its shared memory and stay there for all three passes.  Five
 //    CTAs share an SM, so one CTA's copy and handshake waits overlap the
 //    others' math.
 //  * pass 1: row maxima (packed bf16x2 compares) and sums of 2^(x - max);
@@ -59,6 +59,7 @@ constexpr int kTVCtasPerSm = 4;            // independent CTAs per SM hide each 
 constexpr int kTVChunks = 4;               // bulk copies per row slice (pipelined)
 constexpr int kTVSmemBudget = 52 * 1024;   // bytes of row slices per CTA
 constexpr int kTVMaxW = 256;               // positions per branch held in shared memory
+constexpr int kTVMaxParts = 256;           // (a, s) partials staged in shared memory per round
 constexpr int kTVMaxSlices = 64;           // slices per row (two per lane in one warp)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -117,7 +118,7 @@ template <> struct Vec<float> {
   }
 };
 
-__device__ __forceinline__ float2 ex2_pair(float2 x) { return make_float2(exp2f(x.x), exp2f(x.y)); }
+__device__ __forceinline__ float2 ex2_pair(float2 x) { return make_float2(ex2_fast(x.x), ex2_fast(x.y)); }
 
 __device__ __forceinline__ void warp_lse2(float& m, float& s) {
 #pragma unroll
@@ -138,7 +139,12 @@ struct TVShared {
   float2 red_as[kTVWarps];
   double dred[kTVWarps];
   float sa[kTVMaxW];        // overlaps of the current branch
+  float2 parts[kTVMaxParts];  // (a, s) partials of the current branch's tasks
 };
+// kTVCtasPerSm CTAs must fit the SM's 228 KB of shared memory (1 KB of it
+// reserved per CTA): header + both rows' slices + alignment.
+static_assert(kTVCtasPerSm * (sizeof(TVShared) + 128 + kTVSmemBudget + 1024) <= 228 * 1024,
+              "E2E-TV shared memory does not fit kTVCtasPerSm CTAs per SM");
 
 template <typename Tin, typename Tg>
 __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const TVArgs A) {
@@ -267,8 +273,8 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
           }
         }
         for (int e = e0 + nv * VN + tid; e < e1; e += kTVThreads) {
-          at0.x += exp2f(__fmaf_rn(Elt<Tin>::to_f(st[e]), kLog2e, -mt));
-          ad0.x += exp2f(__fmaf_rn(Elt<Tin>::to_f(sd[e]), kLog2e, -md));
+          at0.x += ex2_fast(__fmaf_rn(Elt<Tin>::to_f(st[e]), kLog2e, -mt));
+          ad0.x += ex2_fast(__fmaf_rn(Elt<Tin>::to_f(sd[e]), kLog2e, -md));
         }
       }
       sum_t = (at0.x + at0.y) + (at1.x + at1.y);
@@ -345,7 +351,7 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
           for (int p = 0; p < VP; ++p) {
             const float2 lt = __ffma2_rn(ft[p], L2E, nLt);
             const float2 ld = __ffma2_rn(fd[p], L2E, nLd);
-            const float2 e = make_float2(exp2f(fminf(lt.x, ld.x)), exp2f(fminf(lt.y, ld.y)));
+            const float2 e = make_float2(ex2_fast(fminf(lt.x, ld.x)), ex2_fast(fminf(lt.y, ld.y)));
             pa2 = __fadd2_rn(pa2, e);
             ps2 = __fadd2_rn(ps2, make_float2(ld.x < lt.x ? e.x : 0.f, ld.y < lt.y ? e.y : 0.f));
           }
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
         for (int e = e0 + nv * VN + tid; e < e1; e += kTVThreads) {
           const float lt = __fmaf_rn(Elt<Tin>::to_f(st[e]), kLog2e, -lse2_t);
           const float ld = __fmaf_rn(Elt<Tin>::to_f(sd[e]), kLog2e, -lse2_d);
-          const float ex = exp2f(fminf(lt, ld));
+          const float ex = ex2_fast(fminf(lt, ld));
           pa2.x += ex;
           ps2.x += (ld < lt) ? ex : 0.f;
         }
@@ -383,19 +389,28 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
     __syncthreads();
     if (need_branch) {
       // Overlap (and this position's s) of every position of the branch,
-      // each summed over its NS slices in a fixed order.
+      // each summed over its NS slices in a fixed order.  The partials of up
+      // to kTVMaxParts / NS positions are loaded in one parallel round trip
+      // into shared memory, then summed there.
       const bool ok = sh.flag != 0;
-      for (int j = tid; j < W; j += kTVThreads) {
-        float av = 0.f, sv = 0.f;
-        for (int cc = 0; cc < NS; ++cc) {
-          const float2 u = __ldcg(&A.part[(size_t)(b * W + j) * NS + cc]);
-          av += u.x;
-          sv += u.y;
+      const int pw = kTVMaxParts / NS;  // positions per round (NS <= kTVMaxSlices)
+      for (int j0 = 0; j0 < W; j0 += pw) {
+        const int j1 = min(W, j0 + pw);
+        for (int k = tid; k < (j1 - j0) * NS; k += kTVThreads)
+          sh.parts[k] = __ldcg(&A.part[((size_t)b * W + j0) * NS + k]);
+        __syncthreads();
+        for (int j = j0 + tid; j < j1; j += kTVThreads) {
+          float av = 0.f, sv = 0.f;
+          for (int cc = 0; cc < NS; ++cc) {
+            const float2 u = sh.parts[(j - j0) * NS + cc];
+            av += u.x;
+            sv += u.y;
+          }
+          sh.sa[j] = ok ? av : qnan;
+          if (j == i) sh.s_own = ok ? sv : qnan;
         }
-        sh.sa[j] = ok ? av : qnan;
-        if (j == i) sh.s_own = ok ? sv : qnan;
+        __syncthreads();
       }
-      __syncthreads();
       if (tid == 0) {
         // g_n = -(1/norm) P_{i-1} S_i, with no division by any overlap
         float P = 1.f;
@@ -494,7 +509,7 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
           for (int e = e0 + nv * VN + tid; e < e1; e += kTVThreads) {
             const float lt = __fmaf_rn(Elt<Tin>::to_f(st[e]), kLog2e, -lse2_t);
             const float ld = __fmaf_rn(Elt<Tin>::to_f(sd[e]), kLog2e, -lse2_d);
-            gout[e] = Elt<Tg>::from_f(exp2f(ld) * ((ld < lt) ? c1 : c0));
+            gout[e] = Elt<Tg>::from_f(ex2_fast(ld) * ((ld < lt) ? c1 : c0));
           }
         }
         // Chunk ch is done by every thread: the next task's copy of it starts.
@@ -522,8 +537,12 @@ void tv_slices(const TVProblem& p, int& NS, int& Lc) {
   const int es = p.logit_dtype == SPECOPD_BF16 ? 2 : 4;
   NS = (int)((2ll * p.V * es + kTVSmemBudget - 1) / kTVSmemBudget);
   if (NS < 1) NS = 1;
-  Lc = (p.V + NS - 1) / NS;
-  Lc = (Lc + 15) / 16 * 16;
+  while (true) {
+    Lc = (p.V + NS - 1) / NS;
+    Lc = (Lc + 15) / 16 * 16;
+    if (2ll * Lc * es <= kTVSmemBudget || Lc == 16) break;
+    ++NS;  // rounding Lc up overshot the budget
+  }
   NS = (p.V + Lc - 1) / Lc;
 }
 

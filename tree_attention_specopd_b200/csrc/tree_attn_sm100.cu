@@ -12,28 +12,32 @@
 //    RT = floor(128 / G) consecutive branch rows of one sequence times the G
 //    query heads of one kv head: M = RT*G <= 128 rows of the MMA.  The rows
 //    of a tile have nearby anchors (anchors are sorted per sequence), so the
-//    trunk keys a tile needs are [0, max anchor]; whole 128-key tiles beyond
+//    trunk keys a tile needs are [0, max anchor]; whole 64-key tiles beyond
 //    the tile's largest anchor are never loaded (masked-tile skipping), and
 //    each row masks only the ragged end of the last tile.
 //  * The branch keys are the tile's own branch nodes (plus the earlier nodes
-//    of its first branch): one or two extra 128-key tiles with the per-row
+//    of its first branch): one or two extra 64-key tiles with the per-row
 //    mask first(branch) <= node <= row.  No dense T x T mask exists anywhere.
 //  * Long trunks are split into key chunks over several CTAs (split-KV);
 //    partial (O, max, sum) go to the workspace and the last CTA of a tile to
 //    finish merges them in a fixed order (no spin-wait, deterministic).
-//  * Per unit, warp 0 drives TMA (Q once, then K/V tiles in a 2-stage ring,
-//    128-byte swizzle), warp 1 issues tcgen05.mma from one thread:
+//  * Two CTAs share an SM (TMEM: 256 of the 512 columns each; shared memory
+//    under half), so one CTA's softmax overlaps the other's MMAs, and one
+//    CTA's prologue and epilogue overlap the other's main loop.
+//  * Per unit, warp 0 drives TMA (Q once, then 64-key K/V tiles in a 2-stage
+//    ring, 128-byte swizzle), warp 1 issues tcgen05.mma from one thread:
 //    S = Q K^T into TMEM (two S buffers, so QK^T of tile j+1 overlaps the
 //    softmax of tile j), and O += P V with P read from TMEM (P overwrites
 //    its S buffer as bf16).  Warps 2-5 own one TMEM lane (= one query row)
-//    each: tcgen05.ld of the S row, mask, online softmax in the log2 domain
-//    with a lazy rescale (O is rescaled in TMEM only when the running max
-//    grows by more than 2^8), tcgen05.st of P.  The epilogue reads O from
-//    TMEM.
+//    each and a full 64-key row of S per tile: tcgen05.ld, mask, online
+//    softmax in the log2 domain with a lazy rescale (O is rescaled in TMEM
+//    only when the running max grows by more than 2^8), tcgen05.st of P.
+//    The epilogue reads O from TMEM 32 columns at a time.
 //  * Every wait is bounded (%globaltimer); expiry sets the status word.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -42,18 +46,20 @@
 namespace specopd {
 namespace sm100 {
 
-constexpr int kThreads = 320;  // warp 0: TMA, warp 1: MMA, warps 2..9: softmax
-constexpr int kBN = 128;       // keys per tile
+constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2..5: softmax + epilogue
+constexpr int kBN = 64;        // keys per tile
 constexpr int kStages = 2;     // K and V ring depth
-constexpr int kTmemCols = 512;
-constexpr int kHalfBytes = 128 * 128;  // one [128 rows x 64 bf16] swizzled box
-constexpr float kRescaleThreshold = 8.f;  // log2 units
+constexpr int kCtasPerSm = 2;
+constexpr int kTmemCols = 256;              // S0 [0,64), S1 [64,128), O [128, 128+D)
+constexpr int kQHalf = 128 * 128;           // Q box: 128 rows x 64 bf16 (swizzled)
+constexpr int kKVHalf = kBN * 128;          // K/V box: 64 rows x 64 bf16 (swizzled)
+constexpr float kRescaleThreshold = 8.f;    // log2 units
 
 struct Params {
   int S, B, W, Hq, Hkv, G, R;
   int RT;              // branch rows per query tile
   int ntile_per_seq, ntile;
-  int nsplit, C;       // key chunks per (tile, kv head), keys per chunk (multiple of 128)
+  int nsplit, C;       // key chunks per (tile, kv head), keys per chunk (multiple of kBN)
   float scale_log2;    // softmax scale * log2(e)
   const int32_t* cu_trunk;
   const int32_t* anchors;
@@ -71,9 +77,7 @@ struct Hdr {
   uint64_t o_done;   // one phase per P.V tile (used by the lazy rescale)
   uint64_t o_final;  // single phase: every MMA of the unit has completed
   uint32_t tmem_base;
-  float red_max[2][2][128];  // [tile parity][column half][row] partial maxima
-  float red_sum[2][128];     // [column half][row] partial sums
-  int kmax;
+  int wmax[4];       // per-warp maxima of the tile's anchors
   int last;
   int abort;
 };
@@ -199,32 +203,41 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, unsigned parit
   return ok;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ------------------------------------------------------------------ kernel
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ktr,
                  const __grid_constant__ CUtensorMap tm_vtr,
                  const __grid_constant__ CUtensorMap tm_kbr,
                  const __grid_constant__ CUtensorMap tm_vbr, const Params P) {
-  constexpr int NH = D / 64;     // 64-column halves of a row
-  constexpr int KSTEPS = D / 16; // MMA K steps of QK^T
+  constexpr int NH = D / 64;      // 64-column halves of a row
+  constexpr int KSTEPS = D / 16;  // MMA K steps of QK^T
+  constexpr int DC = D / 32;      // 32-column chunks of O
   extern __shared__ unsigned char smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sQ = base;
-  uint8_t* sK = sQ + NH * kHalfBytes;
-  uint8_t* sV = sK + kStages * NH * kHalfBytes;
-  Hdr* hdr = reinterpret_cast<Hdr*>(sV + kStages * NH * kHalfBytes);
+  uint8_t* sK = sQ + NH * kQHalf;
+  uint8_t* sV = sK + kStages * NH * kKVHalf;
+  Hdr* hdr = reinterpret_cast<Hdr*>(sV + kStages * NH * kKVHalf);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
-  // ---- work unit: (query tile, kv head, key chunk); heavier tiles first
+  // ---- work unit: (query tile, kv head, key chunk), chunk-major so that the
+  // full leading chunks start first and the partial or empty trailing ones
+  // fill in last; within a chunk, heavier tiles (larger anchors) first.
   const int u = blockIdx.x;
-  const int per_tile = P.Hkv * P.nsplit;
-  const int tile = P.ntile - 1 - u / per_tile;
-  const int c = (u % per_tile) / P.Hkv;
-  const int h = (u % per_tile) % P.Hkv;
+  const int per_c = P.ntile * P.Hkv;
+  const int c = u / per_c;
+  const int tile = P.ntile - 1 - (u % per_c) / P.Hkv;
+  const int h = (u % per_c) % P.Hkv;
   const int s = tile / P.ntile_per_seq;
   const int Wm1 = P.W - 1;
   const int rows_seq = P.B * Wm1;
@@ -232,25 +245,11 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int r1 = min(r0 + P.RT, (s + 1) * rows_seq);
   const int t0 = P.cu_trunk[s];
   const int Ts = P.cu_trunk[s + 1] - t0;
+  const int G = P.G;
+  const int MT = P.RT * G;
 
-  if (tid == 0) hdr->kmax = -1;
-  __syncthreads();
-  for (int r = r0 + tid; r < r1; r += kThreads) {
-    const int a = P.anchors[r / Wm1];
-    if (a >= 0 && a < Ts) atomicMax(&hdr->kmax, a);
-  }
-  __syncthreads();
-  const int kmax = hdr->kmax;
-  const int nact = kmax < 0 ? 1 : (kmax + P.C) / P.C;  // chunks with trunk keys (>= 1)
-  const int k_begin = c * P.C;
-  const int k_end = min(k_begin + P.C, kmax + 1);
-  const int nt = k_end > k_begin ? (k_end - k_begin + kBN - 1) / kBN : 0;
-  if (c > 0 && nt == 0) return;  // nothing for this chunk (uniform over the CTA)
-  const int kb0 = (r0 / Wm1) * Wm1;  // first branch node the tile needs
-  const int nbt = (c == 0) ? (r1 - kb0 + kBN - 1) / kBN : 0;
-  const int nk = nt + nbt;
-
-  // ---- barriers, TMEM
+  // ---- prologue: barriers and the Q copy (thread 0), the tile's largest
+  // valid anchor (warps 0-3), TMEM (warp 1), then one block barrier.
   if (tid == 0) {
     mbar_init(&hdr->q_full, 1);
     for (int i = 0; i < kStages; ++i) {
@@ -261,23 +260,37 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&hdr->s_full[i], 1);
-      mbar_init(&hdr->p_full[i], 256);
+      mbar_init(&hdr->p_full[i], 128);
     }
     mbar_init(&hdr->o_done, 1);
     mbar_init(&hdr->o_final, 1);
     hdr->abort = 0;
     fence_mbar_init();
+    mbar_arrive_expect_tx(&hdr->q_full, (unsigned)(NH * MT * 128));
+    for (int hh = 0; hh < NH; ++hh)
+      tma_load_3d(sQ + hh * kQHalf, &tm_q, hh * 64, h * G, r0, &hdr->q_full);
+  }
+  if (warp < 4) {
+    // RT <= 128: warp w covers rows r0 + 32w .. r0 + 32w + 31
+    const int r = r0 + warp * 32 + lane;
+    int a = -1;
+    if (r < r1) {
+      a = P.anchors[r / Wm1];
+      if (a < 0 || a >= Ts) a = -1;
+    }
+    a = __reduce_max_sync(0xffffffffu, a);
+    if (lane == 0) hdr->wmax[warp] = a;
   }
   // Q rows beyond the tile (M = RT*G < 128) are never written by TMA: zero them.
-  const int MT = P.RT * P.G;
   for (int idx = tid; idx < NH * (128 - MT) * 8; idx += kThreads) {
     const int hh = idx / ((128 - MT) * 8);
     const int rem = idx % ((128 - MT) * 8);
-    reinterpret_cast<uint4*>(sQ + hh * kHalfBytes + (MT + rem / 8) * 128)[rem % 8] =
+    reinterpret_cast<uint4*>(sQ + hh * kQHalf + (MT + rem / 8) * 128)[rem % 8] =
         make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
   if (warp == 1) {
+    __syncwarp();
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&hdr->tmem_base)),
                  "r"(kTmemCols)
@@ -288,30 +301,46 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = hdr->tmem_base;
-  const uint32_t tS[2] = {tmem, tmem + 128};
-  const uint32_t tO = tmem + 256;
+  const int kmax = max(max(hdr->wmax[0], hdr->wmax[1]), max(hdr->wmax[2], hdr->wmax[3]));
+  const int nact = kmax < 0 ? 1 : (kmax + P.C) / P.C;  // chunks with trunk keys (>= 1)
+  const int k_begin = c * P.C;
+  const int k_end = min(k_begin + P.C, kmax + 1);
+  const int nt = k_end > k_begin ? (k_end - k_begin + kBN - 1) / kBN : 0;
+  if (c > 0 && nt == 0) {
+    // Nothing for this chunk (uniform over the CTA).  The Q copy must land
+    // before the CTA's shared memory is released.
+    if (tid == 0 && !mbar_wait(&hdr->q_full, 0)) set_status(SPECOPD_DEV_TIMEOUT);
+    if (warp == 1) {
+      __syncwarp();
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
+    }
+    return;
+  }
+  const int kb0 = (r0 / Wm1) * Wm1;  // first branch node the tile needs
+  const int nbt = (c == 0) ? (r1 - kb0 + kBN - 1) / kBN : 0;
+  const int nk = nt + nbt;
+  const uint32_t tS[2] = {tmem, tmem + kBN};
+  const uint32_t tO = tmem + 2 * kBN;
 
   if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
-      const int G = P.G;
-      mbar_arrive_expect_tx(&hdr->q_full, (unsigned)(NH * MT * 128));
-      for (int hh = 0; hh < NH; ++hh)
-        tma_load_3d(sQ + hh * kHalfBytes, &tm_q, hh * 64, h * G, r0, &hdr->q_full);
       for (int j = 0; j < nk && !hdr->abort; ++j) {
         const int st = j % kStages;
         const bool trunk = j < nt;
         const int row = trunk ? t0 + k_begin + j * kBN : kb0 + (j - nt) * kBN;
         if (j >= kStages && !wait_or_abort(&hdr->k_empty[st], ((j / kStages) - 1) & 1, hdr)) break;
-        mbar_arrive_expect_tx(&hdr->k_full[st], NH * kHalfBytes);
+        mbar_arrive_expect_tx(&hdr->k_full[st], NH * kKVHalf);
         for (int hh = 0; hh < NH; ++hh)
-          tma_load_3d(sK + (st * NH + hh) * kHalfBytes, trunk ? &tm_ktr : &tm_kbr, hh * 64, h,
-                      row, &hdr->k_full[st]);
+          tma_load_3d(sK + (st * NH + hh) * kKVHalf, trunk ? &tm_ktr : &tm_kbr, hh * 64, h, row,
+                      &hdr->k_full[st]);
         if (j >= kStages && !wait_or_abort(&hdr->v_empty[st], ((j / kStages) - 1) & 1, hdr)) break;
-        mbar_arrive_expect_tx(&hdr->v_full[st], NH * kHalfBytes);
+        mbar_arrive_expect_tx(&hdr->v_full[st], NH * kKVHalf);
         for (int hh = 0; hh < NH; ++hh)
-          tma_load_3d(sV + (st * NH + hh) * kHalfBytes, trunk ? &tm_vtr : &tm_vbr, hh * 64, h,
-                      row, &hdr->v_full[st]);
+          tma_load_3d(sV + (st * NH + hh) * kKVHalf, trunk ? &tm_vtr : &tm_vbr, hh * 64, h, row,
+                      &hdr->v_full[st]);
       }
     }
   } else if (warp == 1) {
@@ -328,10 +357,11 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_or_abort(&hdr->p_full[b], (jj >> 1) & 1, hdr)) return false;
         if (!wait_or_abort(&hdr->v_full[st], (jj / kStages) & 1, hdr)) return false;
         tc_fence_after();
+#pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           // B = V tile, MN-major: 16 keys = two 8-row groups of 1024 B; the
-          // 64-column halves of D are kHalfBytes apart.
-          const uint64_t bd = sdesc(v_addr + st * NH * kHalfBytes + kk * 2048, kHalfBytes, 1024);
+          // 64-column halves of D are kKVHalf apart.
+          const uint64_t bd = sdesc(v_addr + st * NH * kKVHalf + kk * 2048, kKVHalf, 1024);
           mma_ts(tO, tS[b] + kk * 8, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&hdr->v_empty[st]);
@@ -345,11 +375,12 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int b = j & 1;
         if (!wait_or_abort(&hdr->k_full[st], (j / kStages) & 1, hdr)) { ok = false; break; }
         tc_fence_after();
+#pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
           // K-major operands: 16 columns = 32 B inside a 128-byte swizzled row.
           const int hh = kk >> 2, w = kk & 3;
-          const uint64_t ad = sdesc(q_addr + hh * kHalfBytes + w * 32, 16, 1024);
-          const uint64_t bd = sdesc(k_addr + (st * NH + hh) * kHalfBytes + w * 32, 16, 1024);
+          const uint64_t ad = sdesc(q_addr + hh * kQHalf + w * 32, 16, 1024);
+          const uint64_t bd = sdesc(k_addr + (st * NH + hh) * kKVHalf + w * 32, 16, 1024);
           mma_ss(tS[b], ad, bd, kIdQK, kk > 0 ? 1u : 0u);
         }
         tc_commit(&hdr->k_empty[st]);
@@ -364,16 +395,11 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else {
     // ================================================================ softmax / epilogue
-    // Eight warps: two per TMEM lane quadrant (warp & 3); the warp's half h2
-    // owns columns [64*h2, 64*h2 + 64) of its 32 rows' S tiles and columns
-    // [DH*h2, DH*h2 + DH) of O.  The two halves of a row exchange their
-    // partial maxima through shared memory once per tile.
-    constexpr int DH = D / 2;
-    const int q4 = warp & 3;             // TMEM lane quadrant of this warp
-    const int h2 = (warp - 2) >> 2;      // column half
-    const int mrow = q4 * 32 + lane;     // query row of the tile = TMEM lane
+    // Warp w accesses TMEM lanes 32*(w%4) .. +31; each thread owns one query
+    // row of the tile (TMEM lane) and all kBN columns of its S tiles.
+    const int q4 = warp & 3;
+    const int mrow = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const int G = P.G;
     const int lr = mrow / G, g = mrow % G;
     const int r = r0 + lr;
     const bool in_tile = (lr < P.RT) && (r < r1);
@@ -387,12 +413,10 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     const bool live = in_tile && !bad;
     const float sl2 = P.scale_log2;
-    const int c0 = 64 * h2;              // first S column of this half
-    float m = -INFINITY, l = 0.f;        // running max (log2 units) and this half's sum
-    uint32_t sv[64];
+    float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum
+    uint32_t sv[kBN];
     // After a wait runs out the warp keeps stepping through the loop with its
-    // TMEM work skipped (dead), so the named barriers shared by the eight
-    // softmax warps still match.
+    // TMEM work skipped (dead).
     bool dead = false;
     for (int j = 0; j < nk; ++j) {
       const int b = j & 1;
@@ -400,12 +424,12 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!dead) {
         tc_fence_after();
         __syncwarp();  // tcgen05.ld/st are warp-collective (.sync.aligned)
-        tmem_ld32(tS[b] + lane_off + c0, sv);
-        tmem_ld32(tS[b] + lane_off + c0 + 32, sv + 32);
+        tmem_ld32(tS[b] + lane_off, sv);
+        tmem_ld32(tS[b] + lane_off + 32, sv + 32);
         tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) sv[e] = 0u;
+        for (int e = 0; e < kBN; ++e) sv[e] = 0u;
       }
       // visible columns of the tile: lo <= col <= hi
       int lo, hi;
@@ -419,24 +443,23 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       if (!live) hi = -1;
       // raw-score maximum (the scale is positive, so it commutes with max)
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (__all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 63)) {
-        // every column of this half is visible to every row of the warp
+      float mx3[3] = {-INFINITY, -INFINITY, -INFINITY};
+      if (__all_sync(0xffffffffu, lo <= 0 && hi >= kBN - 1)) {
+        // every column is visible to every row of the warp
 #pragma unroll
-        for (int e = 0; e < 64; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(sv[e]));
+        for (int e = 0; e + 1 < kBN; e += 2)
+          mx3[(e >> 1) % 3] = fmax3(mx3[(e >> 1) % 3], __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
       } else {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const int col = c0 + e;
-          const float x = (col >= lo && col <= hi) ? __uint_as_float(sv[e]) : -INFINITY;
+        for (int e = 0; e < kBN; ++e) {
+          const float x = (e >= lo && e <= hi) ? __uint_as_float(sv[e]) : -INFINITY;
           sv[e] = __float_as_uint(x);
-          mx4[e & 3] = fmaxf(mx4[e & 3], x);
         }
+#pragma unroll
+        for (int e = 0; e + 1 < kBN; e += 2)
+          mx3[(e >> 1) % 3] = fmax3(mx3[(e >> 1) % 3], __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
       }
-      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      hdr->red_max[b][h2][mrow] = mx;
-      named_bar_sync(1, 256);
-      mx = fmaxf(mx, hdr->red_max[b][h2 ^ 1][mrow]) * sl2;
+      const float mx = fmax3(mx3[0], mx3[1], mx3[2]) * sl2;
       const float m_new = fmaxf(m, mx);
       // Lazy rescale: keep the stale max unless it grew by more than 2^8.
       const bool need = (m != -INFINITY) && (m_new > m + kRescaleThreshold);
@@ -455,117 +478,127 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tc_fence_after();
           __syncwarp();
 #pragma unroll
-          for (int q = 0; q < DH / 32; ++q) {
+          for (int q = 0; q < DC; ++q) {
             uint32_t ov[32];
-            tmem_ld32(tO + lane_off + DH * h2 + q * 32, ov);
+            tmem_ld32(tO + lane_off + q * 32, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-            tmem_st32(tO + lane_off + DH * h2 + q * 32, ov);
+            tmem_st32(tO + lane_off + q * 32, ov);
           }
         }
       }
       // p = 2^(s*scale*log2e - m); masked entries are -inf -> 0
       const float nm = (m == -INFINITY) ? 0.f : -m;
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
+      uint32_t pk[kBN / 2];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float p0 = exp2f(__fmaf_rn(__uint_as_float(sv[2 * e]), sl2, nm));
-        const float p1 = exp2f(__fmaf_rn(__uint_as_float(sv[2 * e + 1]), sl2, nm));
+      for (int e = 0; e < kBN / 2; ++e) {
+        const float p0 = ex2_fast(__fmaf_rn(__uint_as_float(sv[2 * e]), sl2, nm));
+        const float p1 = ex2_fast(__fmaf_rn(__uint_as_float(sv[2 * e + 1]), sl2, nm));
         rs4[e & 3] += p0 + p1;
         pk[e] = pack_bf16x2(p0, p1);
       }
       l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       if (!dead) {
         __syncwarp();
-        tmem_st32(tS[b] + lane_off + 32 * h2, pk);  // P of keys [c0, c0+64) as bf16 pairs
+        tmem_st32(tS[b] + lane_off, pk);  // P of the tile's kBN keys as bf16 pairs
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&hdr->p_full[b]);
       }
     }
     // ---- epilogue
-    float o[DH];
     const bool ok = warp_wait_or_abort(&hdr->o_final, 0, hdr) && !hdr->abort;
     tc_fence_after();
     __syncwarp();
-#pragma unroll
-    for (int q = 0; q < DH / 32; ++q) {
-      uint32_t ov[32];
-      tmem_ld32(tO + lane_off + DH * h2 + q * 32, ov);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) o[q * 32 + e] = __uint_as_float(ov[e]);
-    }
-    // row sum = both halves' partial sums (same reference max)
-    hdr->red_sum[h2][mrow] = l;
-    named_bar_sync(1, 256);
-    l += hdr->red_sum[h2 ^ 1][mrow];
     const int hq = h * G + g;
     const float qnan = __int_as_float(0x7fc00000);
-    auto write_row = [&](const float* acc, float mm, float ll) {
-      __nv_bfloat16* dst = P.out + ((size_t)r * P.Hq + hq) * D + DH * h2;
-      const float inv = (bad || !ok) ? qnan : 1.f / ll;
+    __nv_bfloat16* dst = P.out + ((size_t)r * P.Hq + hq) * D;
+    // 32 columns of the output row as four 16-byte stores
+    auto write_chunk = [&](int q, const float* acc, float inv) {
 #pragma unroll
-      for (int e = 0; e < DH; e += 8) {
+      for (int e = 0; e < 32; e += 8) {
         uint4 v;
         v.x = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
         v.y = pack_bf16x2(acc[e + 2] * inv, acc[e + 3] * inv);
         v.z = pack_bf16x2(acc[e + 4] * inv, acc[e + 5] * inv);
         v.w = pack_bf16x2(acc[e + 6] * inv, acc[e + 7] * inv);
-        *reinterpret_cast<uint4*>(dst + e) = v;
-      }
-      if (h2 == 0) {
-        if (P.lse) P.lse[(size_t)r * P.Hq + hq] = (bad || !ok) ? qnan : (mm + log2f(ll)) * 0.6931471805599453f;
-        if (bad && g == 0) set_status(SPECOPD_DEV_ANCHOR_RANGE);
+        *reinterpret_cast<uint4*>(dst + q * 32 + e) = v;
       }
     };
+    auto write_lse = [&](float mm, float ll) {
+      if (P.lse) P.lse[(size_t)r * P.Hq + hq] = (bad || !ok) ? qnan : (mm + log2f(ll)) * 0.6931471805599453f;
+      if (bad && g == 0) set_status(SPECOPD_DEV_ANCHOR_RANGE);
+    };
     if (nact == 1) {
-      if (in_tile) write_row(o, m, l);
+      const float inv = (bad || !ok) ? qnan : 1.f / l;
+#pragma unroll
+      for (int q = 0; q < DC; ++q) {
+        uint32_t ov[32];
+        tmem_ld32(tO + lane_off + q * 32, ov);
+        tmem_wait_ld();
+        if (in_tile) write_chunk(q, reinterpret_cast<const float*>(ov), inv);
+      }
+      if (in_tile) write_lse(m, l);
     } else {
-      // split-KV: publish this chunk's partial, the last chunk to arrive merges
+      // split-KV: publish this chunk's partial, the last chunk to arrive merges.
+      // Partial layout: float4 k of row mrow at index k * 128 + mrow, so the
+      // 32 rows of a warp store and load 512 contiguous bytes.
       const size_t slot = ((size_t)tile * P.Hkv + h) * P.nsplit;
       const size_t slot_floats = (size_t)128 * D + 256;
-      float* mine = P.part + (slot + c) * slot_floats;
+      float* pbase = P.part + slot * slot_floats;
+      float4* mine4 = reinterpret_cast<float4*>(pbase + c * slot_floats);
 #pragma unroll
-      for (int e = 0; e < DH; e += 4)
-        __stcg(reinterpret_cast<float4*>(mine + (size_t)mrow * D + DH * h2 + e),
-               make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
-      if (h2 == 0) {
-        mine[128 * D + mrow] = m;
-        mine[128 * D + 128 + mrow] = l;
+      for (int q = 0; q < DC; ++q) {
+        uint32_t ov[32];
+        tmem_ld32(tO + lane_off + q * 32, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4)
+          __stcg(mine4 + (q * 8 + e4) * 128 + mrow,
+                 make_float4(__uint_as_float(ov[4 * e4]), __uint_as_float(ov[4 * e4 + 1]),
+                             __uint_as_float(ov[4 * e4 + 2]), __uint_as_float(ov[4 * e4 + 3])));
       }
+      pbase[c * slot_floats + 128 * D + mrow] = m;
+      pbase[c * slot_floats + 128 * D + 128 + mrow] = l;
       __threadfence();
-      named_bar_sync(1, 256);
-      if (mrow == 0 && h2 == 0) {
+      named_bar_sync(1, 128);
+      if (tid == 64) {
         const unsigned old = atomicAdd(&P.cnt[tile * P.Hkv + h], 1u);
         hdr->last = (old == (unsigned)nact - 1u) ? 1 : 0;
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, 128);
       if (hdr->last) {
         __threadfence();
         float mm = -INFINITY;
         for (int cc = 0; cc < nact; ++cc)
-          mm = fmaxf(mm, __ldcg(P.part + (slot + cc) * slot_floats + 128 * D + mrow));
+          mm = fmaxf(mm, __ldcg(pbase + cc * slot_floats + 128 * D + mrow));
         float ll = 0.f;
+        float acc[D];
 #pragma unroll
-        for (int e = 0; e < DH; ++e) o[e] = 0.f;
+        for (int e = 0; e < D; ++e) acc[e] = 0.f;
         for (int cc = 0; cc < nact; ++cc) {
-          const float* pc = P.part + (slot + cc) * slot_floats;
+          const float* pc = pbase + cc * slot_floats;
           const float mc = __ldcg(pc + 128 * D + mrow);
           const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - mm);
           ll += wgt * __ldcg(pc + 128 * D + 128 + mrow);
+          const float4* pc4 = reinterpret_cast<const float4*>(pc);
 #pragma unroll
-          for (int e = 0; e < DH; e += 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(pc + (size_t)mrow * D + DH * h2 + e));
-            o[e] += wgt * v.x;
-            o[e + 1] += wgt * v.y;
-            o[e + 2] += wgt * v.z;
-            o[e + 3] += wgt * v.w;
+          for (int k = 0; k < D / 4; ++k) {
+            const float4 v = __ldcg(pc4 + k * 128 + mrow);
+            acc[4 * k] += wgt * v.x;
+            acc[4 * k + 1] += wgt * v.y;
+            acc[4 * k + 2] += wgt * v.z;
+            acc[4 * k + 3] += wgt * v.w;
           }
         }
-        if (in_tile) write_row(o, mm, ll);
+        if (in_tile) {
+          const float inv = (bad || !ok) ? qnan : 1.f / ll;
+#pragma unroll
+          for (int q = 0; q < DC; ++q) write_chunk(q, acc + q * 32, inv);
+          write_lse(mm, ll);
+        }
       }
     }
   }
@@ -614,43 +647,52 @@ struct Plan {
   size_t part_bytes, cnt_bytes;
 };
 
-Plan make_plan(const AttnProblem& p) {
+// Work decomposition.  base = (query tile, kv head) pairs; each splits into
+// nsplit key chunks of C keys.  With fewer pairs than resident CTA slots
+// (SMs x 2), the smallest nsplit whose units fill every slot once: finer
+// chunks add per-unit prologue, epilogue and merge work.  With one to eight
+// waves of pairs, two chunks halve the tail of the last wave.
+Plan make_plan(const AttnProblem& p, int num_sms) {
   Plan pl;
   pl.RT = 128 / p.G;
   const int rows_seq = p.B * (p.W - 1);
   pl.ntile_per_seq = (rows_seq + pl.RT - 1) / pl.RT;
   pl.ntile = pl.ntile_per_seq * p.S;
   const long long base = (long long)pl.ntile * p.Hkv;
-  int nsplit = 1;
-  if (base < 2 * 148) {
-    nsplit = (int)((2 * 148 + base - 1) / base);
-    const int max_split = std::max(1, p.T_max / 512);
-    if (nsplit > max_split) nsplit = max_split;
-  }
-  int C = (p.T_max + nsplit - 1) / nsplit;
+  const long long slots = (long long)std::max(1, num_sms) * kCtasPerSm;
+  long long want = base < slots ? (slots + base - 1) / base : (base < 8 * slots ? 2 : 1);
+  const int max_split = std::max(1, p.T_max / (4 * kBN));  // chunks of at least 4 key tiles
+  const int best = (int)std::min<long long>(std::min<long long>(want, max_split), 64);
+  int C = (p.T_max + best - 1) / best;
   C = (C + kBN - 1) / kBN * kBN;
-  nsplit = (p.T_max + C - 1) / C;
-  pl.nsplit = nsplit;
+  pl.nsplit = (p.T_max + C - 1) / C;
   pl.C = C;
-  pl.part_bytes = nsplit > 1 ? (size_t)pl.ntile * p.Hkv * nsplit * ((size_t)128 * p.D + 256) * 4 : 0;
+  pl.part_bytes = pl.nsplit > 1 ? (size_t)pl.ntile * p.Hkv * pl.nsplit * ((size_t)128 * p.D + 256) * 4 : 0;
   pl.cnt_bytes = (size_t)pl.ntile * p.Hkv * 4;
   return pl;
 }
 
 size_t smem_bytes(int D) {
   const int NH = D / 64;
-  size_t b = 1024 + (size_t)NH * kHalfBytes * (1 + 2 * kStages) + sizeof(Hdr);
-  // D = 64 would fit two CTAs per SM; each allocates all 512 TMEM columns, so
-  // keep one CTA per SM.
-  if (b < 120 * 1024) b = 120 * 1024;
+  size_t b = 1024 + (size_t)NH * kQHalf + (size_t)2 * kStages * NH * kKVHalf + sizeof(Hdr);
+  // Each CTA allocates half of the SM's TMEM: at most two may be resident.
+  if (b < 80 * 1024) b = 80 * 1024;
   return b;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+    return n;
+  return 148;
 }
 
 }  // namespace
 }  // namespace sm100
 
 size_t attn_sm100_workspace(const AttnProblem& p) {
-  const sm100::Plan pl = sm100::make_plan(p);
+  const sm100::Plan pl = sm100::make_plan(p, sm100::sm_count());
   return ((pl.part_bytes + 255) & ~size_t(255)) + pl.cnt_bytes;
 }
 
@@ -661,7 +703,7 @@ cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_rot, const voi
   using namespace sm100;
   if (p.R == 0) return cudaSuccess;
   if (p.D != 64 && p.D != 128) return cudaErrorInvalidValue;
-  const Plan pl = make_plan(p);
+  const Plan pl = make_plan(p, sm_count());
   const size_t part_off = 0;
   const size_t cnt_off = (pl.part_bytes + 255) & ~size_t(255);
   if (ws_bytes < cnt_off + pl.cnt_bytes) return cudaErrorInvalidValue;
