@@ -33,11 +33,13 @@
 //    position in fixed order -> a_{b,j}, s_n; g_n from the branch.
 //  * pass 3: dz from the slice still in shared memory, chunk by chunk; as
 //    each chunk is done the next task's copy of that chunk starts.
-//  * Tasks are claimed in order with one atomic each.  A CTA claims its next
-//    task only after its own waits are over, so a task never waits for a
-//    task held, unstarted, by the same CTA; with every task of a branch
-//    resident at once (checked on the host: W*NS <= resident CTAs) the
-//    oldest unfinished branch always completes.  Every wait is bounded.
+//  * Static schedule in rounds: the grid is G = k * W * NS resident CTAs and
+//    CTA g runs tasks g, g + G, g + 2G, ...  A round (G consecutive tasks)
+//    therefore holds k whole branches, all of whose tasks start together, so
+//    the handshake waits only absorb the spread of task durations.  A task
+//    waits only for tasks of its own branch, i.e. of its own round, each the
+//    current task of a resident CTA, so every round completes (no deadlock;
+//    the host checks that W*NS CTAs fit at once).  Every wait is bounded.
 //  * The (i = 1, c = 0) task of each branch writes its overlaps and prefix
 //    products; the last branch to finish reduces the loss in a fixed order.
 //  * All math in the log2 domain with packed fp32x2 FMAs: x2 = z*log2(e) -
@@ -81,7 +83,7 @@ struct TVArgs {
   double* bsum;      // [nbranch]
   unsigned* pos_cnt; // [N]      slices of the position with statistics published
   unsigned* br_cnt;  // [nbranch] tasks of the branch with partials published
-  unsigned* ctl;     // [0] claim, [1] branches done, [2] abort
+  unsigned* ctl;     // [1] branches done, [2] abort
 };
 
 // bf16x2 / fp32 vectors of 16 bytes as packed fp32x2 pairs.
@@ -131,7 +133,7 @@ __device__ __forceinline__ void warp_lse2(float& m, float& s) {
 
 struct TVShared {
   uint64_t bar[kTVChunks];  // bulk-copy completion, one phase per task
-  int next;                 // next claimed task
+  int next;                 // next task of this CTA
   int flag;
   float2 lse;               // (lse2_t, lse2_d) of the current position
   float g, s_own;           // gradient coefficient and s_n of the current position
@@ -167,10 +169,12 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
     fence_mbar_init();
   }
 
-  auto claim = [&]() -> int {
-    const int t = (int)atomicAdd(&A.ctl[0], 1u);
-    if (__ldcg(&A.ctl[2]) != 0u) return A.total_tasks;  // a wait ran out: stop
-    return t > A.total_tasks ? A.total_tasks : t;
+  // Next task of this CTA (static rounds); after a wait anywhere ran out,
+  // stop.
+  auto next_task = [&](int t) -> int {
+    if (__ldcg(&A.ctl[2]) != 0u) return A.total_tasks;
+    const long long n = (long long)t + gridDim.x;
+    return n < A.total_tasks ? (int)n : A.total_tasks;
   };
   auto target_row = [&](int n, bool& ok) -> int {
     const int row = A.trow ? A.trow[n] : n;
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
   };
 
   if (tid == 0) {
-    sh.next = claim();
+    sh.next = (int)blockIdx.x < A.total_tasks ? (int)blockIdx.x : A.total_tasks;
     if (sh.next < A.total_tasks && A.aligned) {
       prepare_copy(sh.next);
       for (int ch = 0; ch < kTVChunks; ++ch) issue_chunk(ch);
@@ -454,10 +458,10 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
         }
       }
     }
-    // This task's waits are over: claim the next one (never earlier, so no
-    // task waits for one this CTA holds unstarted).
+    // This task's waits are over: set up the next one, whose copy streams in
+    // chunk by chunk behind the gradient pass.
     if (tid == 0) {
-      sh.next = claim();
+      sh.next = next_task(t);
       if (sh.next < A.total_tasks && A.aligned) prepare_copy(sh.next);
     }
     __syncthreads();
@@ -650,9 +654,11 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
       g_occ_cache[key] = resident;
     }
   }
-  // Every task of a branch must be able to be resident at once.
-  if ((long long)p.W * NS > resident) return cudaErrorInvalidConfiguration;
-  const int grid = std::min(resident, A.total_tasks);
+  // Every task of a branch must be able to be resident at once; the grid is
+  // a whole number of branches' worth of tasks (see the kernel's schedule).
+  const long long wns = (long long)p.W * NS;
+  if (wns > resident) return cudaErrorInvalidConfiguration;
+  const int grid = (int)std::min<long long>(resident / wns * wns, A.total_tasks);
   void* args[] = {&A};
   return cudaLaunchKernel(fn, dim3(grid), dim3(kTVThreads), args, smem, stream);
 }
