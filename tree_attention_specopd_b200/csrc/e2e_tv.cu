@@ -21,13 +21,14 @@
 // exactly that.
 //  * Task = (position n, vocabulary slice c), NS slices per row.  A CTA
 //    (128 threads) holds one task: both rows' slice arrive by 1-D bulk copy
-//    (TMA) into its shared memory and stay there for all three passes.  Five
+//    (TMA) into its shared memory and stay there for all three passes.  Four
 //    CTAs share an SM, so one CTA's copy and handshake waits overlap the
 //    others' math.
-//  * pass 1: row maxima (packed bf16x2 compares) and sums of 2^(x - max);
-//    the slice publishes (max, sum) of both rows and waits (bounded) until
-//    the NS slices of its position have published; every slice combines the
-//    NS statistics in the same fixed order -> identical lse everywhere.
+//  * pass 1: one sweep for row maxima (packed bf16x2 compares) and sums of
+//    2^(x - max) under a running maximum; the slice publishes (max, sum) of
+//    both rows and waits (bounded) until the NS slices of its position have
+//    published; every slice combines the NS statistics in the same fixed
+//    order -> identical lse everywhere.
 //  * pass 2: partial overlap a and masked draft mass s; publish, then wait
 //    until the W*NS tasks of its branch have published; combine per
 //    position in fixed order -> a_{b,j}, s_n; g_n from the branch.
@@ -235,39 +236,39 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
     }
 
     // ------------------------------------------------ pass 1: statistics
-    // Row maxima chunk by chunk as the copies land, then sums of 2^(x - max)
-    // with the same element-to-thread mapping.
+    // One sweep over the slice as the copies land, with the element-to-thread
+    // mapping of passes 2 and 3: per 16-byte group the running maxima (log2
+    // units) move up when the group's maximum exceeds them, and the partial
+    // sums of 2^(x - max) are rescaled then (rarely after the first groups).
     float mt = -INFINITY, md = -INFINITY;
-    for (int ch = 0; ch < kTVChunks; ++ch) {
-      const int e0 = ch * chunk_elems;
-      const int e1 = min(len, e0 + chunk_elems);
-      if (A.aligned && !mbar_wait(&sh.bar[ch], par) && tid == 0) atomicExch(&A.ctl[2], 1u);
-      if (e1 <= e0) continue;
-      const int nv = (e1 - e0) / VN;
-      for (int vi = tid; vi < nv; vi += kTVThreads) {
-        mt = fmaxf(mt, Vec<Tin>::vmax(*reinterpret_cast<const uint4*>(st + e0 + vi * VN)));
-        md = fmaxf(md, Vec<Tin>::vmax(*reinterpret_cast<const uint4*>(sd + e0 + vi * VN)));
-      }
-      for (int e = e0 + nv * VN + tid; e < e1; e += kTVThreads) {
-        mt = fmaxf(mt, Elt<Tin>::to_f(st[e]));
-        md = fmaxf(md, Elt<Tin>::to_f(sd[e]));
-      }
-    }
-    mt *= kLog2e;
-    md *= kLog2e;
     float sum_t = 0.f, sum_d = 0.f;
     {
-      const float2 nmt = make_float2(-mt, -mt), nmd = make_float2(-md, -md);
       float2 at0 = make_float2(0.f, 0.f), at1 = at0, ad0 = at0, ad1 = at0;
+      // Raise a running maximum; a sum formed under a -inf maximum holds only
+      // NaNs from -inf entries and is reset, not rescaled.
+      auto raise = [](float g, float& m, float2& s0, float2& s1) {
+        if (g > m) {
+          const float f = (m == -INFINITY) ? 0.f : ex2_fast(m - g);
+          s0 = (m == -INFINITY) ? make_float2(0.f, 0.f) : __fmul2_rn(s0, make_float2(f, f));
+          s1 = (m == -INFINITY) ? make_float2(0.f, 0.f) : __fmul2_rn(s1, make_float2(f, f));
+          m = g;
+        }
+      };
       for (int ch = 0; ch < kTVChunks; ++ch) {
         const int e0 = ch * chunk_elems;
         const int e1 = min(len, e0 + chunk_elems);
+        if (A.aligned && !mbar_wait(&sh.bar[ch], par) && tid == 0) atomicExch(&A.ctl[2], 1u);
         if (e1 <= e0) continue;
         const int nv = (e1 - e0) / VN;
         for (int vi = tid; vi < nv; vi += kTVThreads) {
+          const uint4 ut = *reinterpret_cast<const uint4*>(st + e0 + vi * VN);
+          const uint4 ud = *reinterpret_cast<const uint4*>(sd + e0 + vi * VN);
+          raise(Vec<Tin>::vmax(ut) * kLog2e, mt, at0, at1);
+          raise(Vec<Tin>::vmax(ud) * kLog2e, md, ad0, ad1);
           float2 ft[VP], fd[VP];
-          Vec<Tin>::pairs(*reinterpret_cast<const uint4*>(st + e0 + vi * VN), ft);
-          Vec<Tin>::pairs(*reinterpret_cast<const uint4*>(sd + e0 + vi * VN), fd);
+          Vec<Tin>::pairs(ut, ft);
+          Vec<Tin>::pairs(ud, fd);
+          const float2 nmt = make_float2(-mt, -mt), nmd = make_float2(-md, -md);
 #pragma unroll
           for (int p = 0; p < VP; p += 2) {
             at0 = __fadd2_rn(at0, ex2_pair(__ffma2_rn(ft[p], L2E, nmt)));
@@ -277,8 +278,12 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
           }
         }
         for (int e = e0 + nv * VN + tid; e < e1; e += kTVThreads) {
-          at0.x += ex2_fast(__fmaf_rn(Elt<Tin>::to_f(st[e]), kLog2e, -mt));
-          ad0.x += ex2_fast(__fmaf_rn(Elt<Tin>::to_f(sd[e]), kLog2e, -md));
+          const float xt = Elt<Tin>::to_f(st[e]) * kLog2e;
+          const float xd = Elt<Tin>::to_f(sd[e]) * kLog2e;
+          raise(xt, mt, at0, at1);
+          raise(xd, md, ad0, ad1);
+          at0.x += ex2_fast(xt - mt);
+          ad0.x += ex2_fast(xd - md);
         }
       }
       sum_t = (at0.x + at0.y) + (at1.x + at1.y);
