@@ -74,6 +74,8 @@ typedef enum { SPECOPD_F32 = 0, SPECOPD_BF16 = 1 } specopd_dtype;
 #define SPECOPD_DEV_ROW_RANGE 0x2u     /* a target_row outside [0, rows_target) */
 #define SPECOPD_DEV_ALL_NEG_INF 0x4u   /* a logit row with no finite entry      */
 #define SPECOPD_DEV_TIMEOUT 0x8u       /* a bounded wait ran out                */
+#define SPECOPD_DEV_LAYOUT 0x10u       /* shared memory not laid out as the kernel
+                                          requires; the kernel wrote nothing    */
 
 /* Human-readable name of a status code.  Never NULL. */
 const char* specopd_status_string(int status);

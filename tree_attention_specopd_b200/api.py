@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libspecopd.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "specopd.h")
 
 F32, BF16 = 0, 1
-DEV_ANCHOR_RANGE, DEV_ROW_RANGE, DEV_ALL_NEG_INF, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+DEV_ANCHOR_RANGE, DEV_ROW_RANGE, DEV_ALL_NEG_INF, DEV_TIMEOUT, DEV_LAYOUT = 0x1, 0x2, 0x4, 0x8, 0x10
 
 _STATUS = {0: "SPECOPD_OK", 1: "SPECOPD_ERR_INVALID_ARG", 2: "SPECOPD_ERR_UNSUPPORTED",
            3: "SPECOPD_ERR_WORKSPACE", 4: "SPECOPD_ERR_CUDA", 5: "SPECOPD_ERR_TIMEOUT",

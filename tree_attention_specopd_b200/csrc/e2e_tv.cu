@@ -645,6 +645,9 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
     // The attribute is per function: set it on every launch (another problem
     // size may have lowered it since).
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     auto key = std::make_tuple(dev, fn, (int)smem);
     auto it = g_occ_cache.find(key);

@@ -48,7 +48,8 @@ namespace sm100 {
 
 constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2..5: softmax + epilogue
 constexpr int kBN = 64;        // keys per tile
-constexpr int kStages = 2;     // K and V ring depth
+constexpr int kKStages = 3;    // K ring depth (K tiles run ahead of V tiles)
+constexpr int kVStages = 2;    // V ring depth
 constexpr int kCtasPerSm = 2;
 constexpr int kTmemCols = 256;              // S0 [0,64), S1 [64,128), O [128, 128+D)
 constexpr int kQHalf = 128 * 128;           // Q box: 128 rows x 64 bf16 (swizzled)
@@ -71,8 +72,8 @@ struct Params {
 
 struct Hdr {
   uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_done;   // one phase per P.V tile (used by the lazy rescale)
   uint64_t o_final;  // single phase: every MMA of the unit has completed
@@ -219,13 +220,18 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   constexpr int NH = D / 64;      // 64-column halves of a row
   constexpr int KSTEPS = D / 16;  // MMA K steps of QK^T
   constexpr int DC = D / 32;      // 32-column chunks of O
-  extern __shared__ unsigned char smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* sQ = base;
+  // 128-byte swizzled tiles need 1024-byte aligned shared memory; the
+  // dynamic region starts at the CTA's shared-memory base (no static shared
+  // memory), and two CTAs per SM leave no room for alignment slack.
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  uint8_t* sQ = smem_raw;
   uint8_t* sK = sQ + NH * kQHalf;
-  uint8_t* sV = sK + kStages * NH * kKVHalf;
-  Hdr* hdr = reinterpret_cast<Hdr*>(sV + kStages * NH * kKVHalf);
+  uint8_t* sV = sK + kKStages * NH * kKVHalf;
+  Hdr* hdr = reinterpret_cast<Hdr*>(sV + kVStages * NH * kKVHalf);
+  if (smem_u32(smem_raw) & 1023u) {  // uniform over the CTA; nothing touched yet
+    if (threadIdx.x == 0) set_status(SPECOPD_DEV_LAYOUT);
+    return;
+  }
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -252,9 +258,11 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   // valid anchor (warps 0-3), TMEM (warp 1), then one block barrier.
   if (tid == 0) {
     mbar_init(&hdr->q_full, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&hdr->k_full[i], 1);
       mbar_init(&hdr->k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&hdr->v_full[i], 1);
       mbar_init(&hdr->v_empty[i], 1);
     }
@@ -327,20 +335,28 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
-      for (int j = 0; j < nk && !hdr->abort; ++j) {
-        const int st = j % kStages;
-        const bool trunk = j < nt;
-        const int row = trunk ? t0 + k_begin + j * kBN : kb0 + (j - nt) * kBN;
-        if (j >= kStages && !wait_or_abort(&hdr->k_empty[st], ((j / kStages) - 1) & 1, hdr)) break;
-        mbar_arrive_expect_tx(&hdr->k_full[st], NH * kKVHalf);
-        for (int hh = 0; hh < NH; ++hh)
-          tma_load_3d(sK + (st * NH + hh) * kKVHalf, trunk ? &tm_ktr : &tm_kbr, hh * 64, h, row,
-                      &hdr->k_full[st]);
-        if (j >= kStages && !wait_or_abort(&hdr->v_empty[st], ((j / kStages) - 1) & 1, hdr)) break;
-        mbar_arrive_expect_tx(&hdr->v_full[st], NH * kKVHalf);
-        for (int hh = 0; hh < NH; ++hh)
-          tma_load_3d(sV + (st * NH + hh) * kKVHalf, trunk ? &tm_vtr : &tm_vbr, hh * 64, h, row,
-                      &hdr->v_full[st]);
+      // K tiles run kKStages - kVStages tiles ahead of V tiles: the QK^T that
+      // frees a K slot completes before the P.V that frees the V slot of the
+      // same tile, so a blocked V copy never holds back the next K copy.
+      auto row_of = [&](int j) { return j < nt ? t0 + k_begin + j * kBN : kb0 + (j - nt) * kBN; };
+      constexpr int kLead = kKStages - kVStages;
+      for (int i = 0; i < nk + kLead && !hdr->abort; ++i) {
+        if (i < nk) {
+          const int j = i, st = j % kKStages;
+          if (j >= kKStages && !wait_or_abort(&hdr->k_empty[st], ((j / kKStages) - 1) & 1, hdr)) break;
+          mbar_arrive_expect_tx(&hdr->k_full[st], NH * kKVHalf);
+          for (int hh = 0; hh < NH; ++hh)
+            tma_load_3d(sK + (st * NH + hh) * kKVHalf, j < nt ? &tm_ktr : &tm_kbr, hh * 64, h,
+                        row_of(j), &hdr->k_full[st]);
+        }
+        if (i >= kLead) {
+          const int j = i - kLead, st = j % kVStages;
+          if (j >= kVStages && !wait_or_abort(&hdr->v_empty[st], ((j / kVStages) - 1) & 1, hdr)) break;
+          mbar_arrive_expect_tx(&hdr->v_full[st], NH * kKVHalf);
+          for (int hh = 0; hh < NH; ++hh)
+            tma_load_3d(sV + (st * NH + hh) * kKVHalf, j < nt ? &tm_vtr : &tm_vbr, hh * 64, h,
+                        row_of(j), &hdr->v_full[st]);
+        }
       }
     }
   } else if (warp == 1) {
@@ -353,9 +369,9 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const uint32_t v_addr = smem_u32(sV);
       auto pv = [&](int jj) -> bool {
         const int b = jj & 1;
-        const int st = jj % kStages;
+        const int st = jj % kVStages;
         if (!wait_or_abort(&hdr->p_full[b], (jj >> 1) & 1, hdr)) return false;
-        if (!wait_or_abort(&hdr->v_full[st], (jj / kStages) & 1, hdr)) return false;
+        if (!wait_or_abort(&hdr->v_full[st], (jj / kVStages) & 1, hdr)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
@@ -371,9 +387,9 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       bool ok = wait_or_abort(&hdr->q_full, 0, hdr);
       tc_fence_after();
       for (int j = 0; j < nk && ok; ++j) {
-        const int st = j % kStages;
+        const int st = j % kKStages;
         const int b = j & 1;
-        if (!wait_or_abort(&hdr->k_full[st], (j / kStages) & 1, hdr)) { ok = false; break; }
+        if (!wait_or_abort(&hdr->k_full[st], (j / kKStages) & 1, hdr)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -674,7 +690,7 @@ Plan make_plan(const AttnProblem& p, int num_sms) {
 
 size_t smem_bytes(int D) {
   const int NH = D / 64;
-  size_t b = 1024 + (size_t)NH * kQHalf + (size_t)2 * kStages * NH * kKVHalf + sizeof(Hdr);
+  size_t b = (size_t)NH * kQHalf + (size_t)(kKStages + kVStages) * NH * kKVHalf + sizeof(Hdr);
   // Each CTA allocates half of the SM's TMEM: at most two may be resident.
   if (b < 80 * 1024) b = 80 * 1024;
   return b;
@@ -732,10 +748,16 @@ cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_rot, const voi
   const dim3 grid((unsigned)((size_t)pl.ntile * p.Hkv * pl.nsplit));
   if (p.D == 128) {
     e = cudaFuncSetAttribute(tree_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tree_attn_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     tree_attn_kernel<128><<<grid, kThreads, smem, st>>>(tq, tktr, tvtr, tkbr, tvbr, P);
   } else {
     e = cudaFuncSetAttribute(tree_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tree_attn_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     tree_attn_kernel<64><<<grid, kThreads, smem, st>>>(tq, tktr, tvtr, tkbr, tvbr, P);
   }
