@@ -37,7 +37,16 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-WORKLOAD = "8b"
+WORKLOAD = "8b"  # default; --workload selects another of the synthetic configs
+WORKLOAD_NAMES = {
+    "tiny": "tiny fp32: T=256, B=4, W=4, 4q/1kv heads, head_dim 64, vocab 1024, N=16 positions",
+    "8b": "8B-shaped single layer: T=4096, B=64 anchors, W=8, 32q/8kv heads, head_dim 128, "
+          "vocab 151936, N=512 positions",
+    "long": "long trunk: T=32768, B=256 anchors, W=16, 40q/8kv heads, head_dim 128, vocab 151936, "
+            "N=4096 positions",
+    "packed": "packed batch: 8 sequences of 2048-16384 tokens, B=128 anchors each, W=16, "
+              "64q/8kv heads, head_dim 128, vocab 248320, N=16384 positions",
+}
 METRIC = "scored branch rows/s (tree-attn + E2E-TV); % of bf16 TC peak and HBM roofline"
 
 
@@ -98,17 +107,19 @@ def _clock_summary(path, dev_index):
 # ------------------------------------------------------------------ device problem
 
 class Problem:
-    """Device-resident inputs and outputs of one step (the 8B-shaped workload)."""
+    """Device-resident inputs and outputs of one step of a named workload."""
 
-    def __init__(self, torch, api, dev, seed_offset=0):
+    def __init__(self, torch, api, dev, seed_offset=0, workload=WORKLOAD):
         self.torch, self.api, self.dev = torch, api, dev
-        acfg = synth.attn_config(WORKLOAD)
-        tcfg = synth.tv_config(WORKLOAD)
+        acfg = synth.attn_config(workload)
+        tcfg = synth.tv_config(workload)
         self.acfg, self.tcfg = acfg, tcfg
         inp = synth.attention_inputs(acfg)
         self.inp = inp
-        bf = torch.bfloat16
-        t = lambda x: torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev).to(bf)  # noqa
+        adt = torch.bfloat16 if acfg.dtype == "bf16" else torch.float32
+        ldt = torch.bfloat16 if tcfg.dtype == "bf16" else torch.float32
+        bf = ldt
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev).to(adt)  # noqa
         self.cu_host = [int(c) for c in inp.cu_trunk]
         self.cu_dev = torch.tensor(inp.cu_trunk, device=dev)
         self.anchors = torch.tensor(inp.anchors, device=dev)
@@ -126,7 +137,7 @@ class Problem:
                                self.score_row)
         # trunk K cache, rotated once (trunk prefill)
         api.specopd_rope_apply(self.k_tr, self.sem_pos[: self.T_tot].contiguous(), acfg.rope_base)
-        self.desc = api.attn_desc(S, B, W, acfg.Hq, acfg.Hkv, acfg.D, "bf16", acfg.rope_base)
+        self.desc = api.attn_desc(S, B, W, acfg.Hq, acfg.Hkv, acfg.D, acfg.dtype, acfg.rope_base)
         ws = api.specopd_tree_attn_workspace_size(self.desc, self.cu_host)
         self.attn_ws = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.out = torch.empty_like(self.q_br)
@@ -141,18 +152,21 @@ class Problem:
         rows_t = self.T_tot + self.R
         self.rows_t = rows_t
         self.z_t = torch.zeros((rows_t, V), dtype=bf, device=dev)
-        zt = torch.randn((self.N, V), generator=g, device=dev) * tcfg.sigma_t
-        k = torch.randint(1, 4, (self.N,), generator=g, device=dev)
-        ids = torch.randint(0, V, (self.N, 3), generator=g, device=dev)
-        bump = (torch.arange(3, device=dev)[None, :] < k[:, None]).float() * tcfg.bump
-        zt.scatter_add_(1, ids, bump)
-        zd = zt + torch.randn((self.N, V), generator=g, device=dev) * tcfg.sigma_d
-        torch.cuda.synchronize()
+        self.z_d = torch.empty((self.N, V), dtype=bf, device=dev)
         sr = self.score_row.long()
-        self.z_t[sr] = zt.to(bf)
-        self.z_d = zd.to(bf)
-        del zt, zd
-        self.tdesc = api.tv_desc(S * B, W, V, rows_t, "bf16", "f32", True,
+        for n0 in range(0, self.N, 2048):  # row chunks bound the fp32 temporaries
+            n1 = min(self.N, n0 + 2048)
+            zt = torch.randn((n1 - n0, V), generator=g, device=dev) * tcfg.sigma_t
+            k = torch.randint(1, 4, (n1 - n0,), generator=g, device=dev)
+            ids = torch.randint(0, V, (n1 - n0, 3), generator=g, device=dev)
+            bump = (torch.arange(3, device=dev)[None, :] < k[:, None]).float() * tcfg.bump
+            zt.scatter_add_(1, ids, bump)
+            zd = zt + torch.randn((n1 - n0, V), generator=g, device=dev) * tcfg.sigma_d
+            self.z_t[sr[n0:n1]] = zt.to(bf)
+            self.z_d[n0:n1] = zd.to(bf)
+            del zt, zd
+        torch.cuda.synchronize()
+        self.tdesc = api.tv_desc(S * B, W, V, rows_t, tcfg.dtype, "f32", True,
                                  norm_count=self.N)
         self.tv_ws = torch.empty(api.specopd_e2e_tv_workspace_size(self.tdesc), dtype=torch.uint8,
                                  device=dev)
@@ -163,7 +177,8 @@ class Problem:
         self.numer = torch.empty(1, dtype=torch.float64, device=dev)
         self.grad = torch.empty((self.N, V), dtype=f32, device=dev)
         self.flops = attention_flops(acfg, inp.anchors)
-        self.tv_bytes = float(self.N) * V * (2 + 2 + 4)
+        es = 2 if tcfg.dtype == "bf16" else 4
+        self.tv_bytes = float(self.N) * V * (2 * es + 4)
 
     def step(self, ev=None):
         api, acfg = self.api, self.acfg
@@ -202,13 +217,14 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     api.load()
-    pb = Problem(torch, api, dev, seed_offset=rank)
+    wl = args.workload
+    pb = Problem(torch, api, dev, seed_offset=rank, workload=wl)
     # Distributed normalisation: every rank's gradient and loss divide by the
     # GLOBAL position count (gathered once), and the prefix-product sums are
     # all-reduced after each step.
     n_global = sdist.global_count(pb.N, device=dev)
     if world > 1:
-        pb.tdesc = api.tv_desc(pb.acfg.S * pb.acfg.B, pb.acfg.W, pb.V, pb.rows_t, "bf16", "f32",
+        pb.tdesc = api.tv_desc(pb.acfg.S * pb.acfg.B, pb.acfg.W, pb.V, pb.rows_t, pb.tcfg.dtype, "f32",
                                True, norm_count=n_global)
     numer_all = torch.zeros(1, dtype=torch.float64, device=dev)
     loss_all = torch.zeros(1, dtype=torch.float64, device=dev)
@@ -260,8 +276,9 @@ def run_gpu(args):
     if st != 0:
         raise RuntimeError(f"device status {st:#x} after the timed steps")
 
-    # ---- end-to-end through the public API with host buffers
-    e2e = e2e_measure(torch, api, pb, args, dev, world)
+    # ---- end-to-end through the public API with host buffers (the default
+    # workload; the larger ones would copy tens of GB per step)
+    e2e = e2e_measure(torch, api, pb, args, dev, world) if wl == WORKLOAD else None
 
     if rank == 0:
         peaks = _peaks()
@@ -282,22 +299,26 @@ def run_gpu(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16",
+            "dtype": pb.acfg.dtype,
             "data": "synthetic",
-            "config": {"workload": "8B-shaped single layer: T=4096, B=64 anchors, W=8, 32q/8kv "
-                                   "heads, head_dim 128, vocab 151936, N=512 positions",
+            "config": {"workload": WORKLOAD_NAMES[wl],
                        "rows_per_step_per_gpu": pb.R, "positions_per_step_per_gpu": pb.N,
                        "parallelism": f"dp{world} (branch batches per rank)",
-                       "l2": "inputs larger than L2 (0.31 GB of logits read per step vs 126 MB)"},
+                       "l2": (f"inputs larger than L2 ({pb.tv_bytes / 2e9:.2f} GB of logits read "
+                              "per step vs 126 MB)") if pb.tv_bytes / 2 > 126e6 else
+                             "inputs fit in L2 (small workload; not an HBM measurement)"},
             "supervised_tokens_per_s": pb.N * world / (ms_step / 1e3),
             "roofline": {"bound": "hbm", "kernel": "e2e_tv", "achieved": tv_gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": tv_gbs / peaks["hbm_gbs"], "traffic": traffic,
                          "algorithmic_bytes_per_launch": pb.tv_bytes, "launch_ms": tv_ms,
                          "peak_src": peaks["src"]},
-            "attention_roofline": {"bound": "tensor", "kernel": "tree_attn", "achieved": attn_tflops,
-                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                   "frac": attn_tflops / peaks["bf16_tflops"],
+            "attention_roofline": {"bound": "tensor" if pb.acfg.dtype == "bf16" else "fp32 SIMT",
+                                   "kernel": "tree_attn", "achieved": attn_tflops,
+                                   "peak": peaks["bf16_tflops"] if pb.acfg.dtype == "bf16" else None,
+                                   "unit": "TFLOP/s",
+                                   "frac": attn_tflops / peaks["bf16_tflops"]
+                                   if pb.acfg.dtype == "bf16" else None,
                                    "algorithmic_flops_per_launch": pb.flops, "launch_ms": attn_ms,
                                    "peak_src": peaks["src"]},
             "loss": loss,
@@ -305,19 +326,38 @@ def run_gpu(args):
             "e2e": e2e,
             "gpu_launches": KERNELS_PER_STEP * args.steps,
         }
+        if e2e is None:
+            line["e2e_note"] = "host-buffer end-to-end measured on the default 8B workload only"
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds, workload=wl)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
 
 
+TV_SOURCES = ("tree_attention_specopd_b200/csrc/e2e_tv.cu", "tree_attention_specopd_b200/csrc/common.cuh")
+
+
+def tv_source_sha256():
+    """Hash of the E2E-TV kernel sources (the counters below belong to it)."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TV_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def _ncu_traffic():
-    """DRAM bytes per e2e_tv launch from a committed ncu summary, if present."""
+    """DRAM bytes per e2e_tv launch from the committed ncu summary, or None
+    when it is absent or was taken on other kernel sources."""
     path = os.path.join(ROOT, "profiles", "e2e_tv_8b_traffic.json")
     try:
-        return json.load(open(path))["dram_bytes_per_launch"]
+        rec = json.load(open(path))
+        if rec.get("source_sha256") != tv_source_sha256():
+            return None
+        return rec["dram_bytes_per_launch"]
     except Exception:
         return None
 
@@ -371,14 +411,14 @@ def e2e_measure(torch, api, pb, args, dev, world):
 
 # ------------------------------------------------------------------ CPU oracle
 
-def cpu_baseline(seconds=15.0, nbranch=None):
+def cpu_baseline(seconds=15.0, nbranch=None, workload=WORKLOAD):
     """The fp64 oracle, as it stands, on a bounded sample of the workload:
     whole branches (their W-1 attention rows and W TV positions), timed on
     the host cores; reported in the bench's unit (scored rows/s)."""
     from oracle import attention as oatt
     from oracle import tv as otv
-    acfg = synth.attn_config(WORKLOAD)
-    tcfg = synth.tv_config(WORKLOAD)
+    acfg = synth.attn_config(workload)
+    tcfg = synth.tv_config(workload)
     inp = synth.attention_inputs(acfg)
     rows = 0
     t0 = time.perf_counter()
@@ -403,7 +443,7 @@ def cpu_baseline(seconds=15.0, nbranch=None):
     except Exception:
         threads = os.cpu_count()
     return {"value": rows / el, "unit": "rows/s", "cores": threads, "kind": "oracle",
-            "sample": f"{b} of {acfg.B} branches of the 8B-shaped workload "
+            "sample": f"{b} of {acfg.S * acfg.B} branches of the {workload} workload "
                       f"({rows} rows, {b * acfg.W} TV positions) in {el:.1f} s; "
                       f"host has {os.cpu_count()} cores"}
 
@@ -413,13 +453,15 @@ def run_reference(args):
     if rank != 0:
         return
     per = []
+    wl = args.workload
+    W = synth.attn_config(wl).W
     for _ in range(args.warmup):
-        cpu_baseline(nbranch=1)
+        cpu_baseline(nbranch=1, workload=wl)
     t0 = time.perf_counter()
     rows = 0
     for _ in range(args.steps):
-        r = cpu_baseline(nbranch=1)
-        rows += 7
+        r = cpu_baseline(nbranch=1, workload=wl)
+        rows += W - 1
         per.append(r)
     el = time.perf_counter() - t0
     value = rows / el
@@ -428,10 +470,11 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": "8B-shaped single layer (one branch of it per step)"},
+            "config": {"workload": WORKLOAD_NAMES[wl] + " (one branch of it per step)"},
             "cpu_baseline": {"value": value, "unit": "rows/s", "kind": "oracle",
                              "cores": per[-1]["cores"] if per else os.cpu_count(),
-                             "sample": "1 branch (7 attention rows, 8 TV positions) per step"},
+                             "sample": f"1 branch ({W - 1} attention rows, {W} TV positions) "
+                                       "per step"},
             "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -445,6 +488,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOAD_NAMES),
+                    help="synthetic configuration (default: the 8B-shaped one)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

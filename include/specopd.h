@@ -268,7 +268,7 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* desc,
  * every GPU that loads the library until the process exits.
  *   - Size limit: returns SPECOPD_ERR_WORKSPACE, launching nothing, when
  *     specopd_e2e_tv_workspace_size(desc) exceeds the array (8 MiB: about
- *     30,000 positions at a 151,936-token bf16 vocabulary).
+ *     28,000 positions at a 151,936-token bf16 vocabulary and W = 8).
  *   - The first call on each device resolves the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - All calls on a device share the array, which keeps the last call's

@@ -29,7 +29,7 @@ def _read_fixture(name):
 
 
 def test_worked_example_fixture():
-    # Review §3.1 example ("Enjoy a quiet evening at home", anchors a, evening).
+    # Review §3.1 worked example: a six-token reference, anchors at tokens 1 and 3.
     fx = _read_fixture("tree_enjoy_example.txt")
     parent, sem_pos, score_row = tree.tree_build(fx["cu_trunk"], fx["anchors"],
                                                  fx["B"][0], fx["W"][0])

@@ -34,13 +34,15 @@
 //    position in fixed order -> a_{b,j}, s_n; g_n from the branch.
 //  * pass 3: dz from the slice still in shared memory, chunk by chunk; as
 //    each chunk is done the next task's copy of that chunk starts.
-//  * Static schedule in rounds: the grid is G = k * W * NS resident CTAs and
-//    CTA g runs tasks g, g + G, g + 2G, ...  A round (G consecutive tasks)
-//    therefore holds k whole branches, all of whose tasks start together, so
-//    the handshake waits only absorb the spread of task durations.  A task
-//    waits only for tasks of its own branch, i.e. of its own round, each the
-//    current task of a resident CTA, so every round completes (no deadlock;
-//    the host checks that W*NS CTAs fit at once).  Every wait is bounded.
+//  * Static schedule in rounds: CTA g of a grid of G resident CTAs runs
+//    tasks g, g + G, g + 2G, ...  G is a multiple of W*NS when that idles
+//    few slots: a round (G consecutive tasks) then holds whole branches,
+//    all of whose tasks start together, so the handshake waits only absorb
+//    the spread of task durations.  Deadlock freedom needs only G >= W*NS
+//    (checked on the host): a task waits for tasks of its own branch, less
+//    than W*NS ids away, and a task not yet started is held by a CTA busy
+//    with the task G ids before it, so a cycle of waits would have to gain
+//    G ids per step while moving fewer than W*NS.  Every wait is bounded.
 //  * The (i = 1, c = 0) task of each branch writes its overlaps and prefix
 //    products; the last branch to finish reduces the loss in a fixed order.
 //  * All math in the log2 domain with packed fp32x2 FMAs: x2 = z*log2(e) -
@@ -662,11 +664,14 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
       g_occ_cache[key] = resident;
     }
   }
-  // Every task of a branch must be able to be resident at once; the grid is
-  // a whole number of branches' worth of tasks (see the kernel's schedule).
+  // Every task of a branch must be able to be resident at once.  The grid is
+  // a whole number of branches' worth of tasks when that idles under 5 % of
+  // the resident slots, else every slot (see the kernel's schedule).
   const long long wns = (long long)p.W * NS;
   if (wns > resident) return cudaErrorInvalidConfiguration;
-  const int grid = (int)std::min<long long>(resident / wns * wns, A.total_tasks);
+  const long long spare = resident % wns;
+  const long long G = spare * 20 <= resident ? resident - spare : resident;
+  const int grid = (int)std::min<long long>(G, A.total_tasks);
   void* args[] = {&A};
   return cudaLaunchKernel(fn, dim3(grid), dim3(kTVThreads), args, smem, stream);
 }
