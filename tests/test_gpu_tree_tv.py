@@ -230,7 +230,8 @@ def test_tv_8b_bf16_through_score_rows(lib):
     (1003, 2, 3, "bf16", "bf16"),  # odd row stride in bf16, bf16 grads
     (4096, 1, 7, "bf16", "f32"),   # W = 1
     (1000, 3, 4, "f32", "bf16"),   # fp32 logits, bf16 gradient (aligned path)
-    (111_104, 4, 2, "bf16", "f32"),  # cluster of 3 CTAs, ragged last slice, aligned path
+    (111_104, 4, 2, "bf16", "f32"),  # ragged last slice, aligned path
+    (40_000, 64, 2, "bf16", "f32"),  # W*NS = 256 tasks per branch, rounds of whole branches
 ])
 def test_tv_shapes(lib, V, W, nb, dtype, gdt):
     rng = np.random.default_rng(V + W)
