@@ -543,8 +543,9 @@ struct TVLayout {
   size_t stats, part, bsum, pos_cnt, br_cnt, ctl, total, zero_begin, zero_bytes;
 };
 
-// Slice geometry: NS slices of Lc elements (a multiple of 16) per row.
-void tv_slices(const TVProblem& p, int& NS, int& Lc) {
+// Slice geometry: the fewest slices per row, NS slices of Lc elements (a
+// multiple of 16), whose two rows fit the shared-memory budget.
+void tv_min_slices(const TVProblem& p, int& NS, int& Lc) {
   const int es = p.logit_dtype == SPECOPD_BF16 ? 2 : 4;
   NS = (int)((2ll * p.V * es + kTVSmemBudget - 1) / kTVSmemBudget);
   if (NS < 1) NS = 1;
@@ -557,10 +558,39 @@ void tv_slices(const TVProblem& p, int& NS, int& Lc) {
   NS = (p.V + Lc - 1) / Lc;
 }
 
-TVLayout tv_layout(const TVProblem& p) {
+// Slice count for `resident` co-resident CTAs: from the budget's count up,
+// the first for which rounds of whole branches (multiples of W*NS CTAs)
+// idle under 5 % of the resident CTAs; the budget's count if none does.  A
+// round then holds whole branches (see the kernel's schedule); a branch that
+// straddles two rounds makes its early tasks wait about a whole task.
+void tv_slices(const TVProblem& p, long long resident, int& NS, int& Lc) {
+  tv_min_slices(p, NS, Lc);
+  for (int want = NS; want <= kTVMaxSlices; ++want) {
+    int lc = (p.V + want - 1) / want;
+    lc = (lc + 15) / 16 * 16;
+    const int ns = (p.V + lc - 1) / lc;
+    const long long wns = (long long)p.W * ns;
+    if (ns > kTVMaxSlices || wns > resident) break;
+    if ((resident % wns) * 20 <= resident) {
+      NS = ns;
+      Lc = lc;
+      return;
+    }
+  }
+}
+
+// Resident CTAs assumed for host-side sizing: the current device's SMs (148
+// without one) times kTVCtasPerSm.
+long long nominal_resident() {
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+    nsm = 148;
+  return (long long)nsm * kTVCtasPerSm;
+}
+
+TVLayout tv_layout(const TVProblem& p, int NS) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  int NS, Lc;
-  tv_slices(p, NS, Lc);
   TVLayout L;
   size_t off = 0;
   L.stats = off;   off = up(off + sizeof(float4) * (size_t)p.N * NS);
@@ -594,25 +624,64 @@ std::map<std::tuple<int, void*, int>, int> g_occ_cache;  // (dev, fn, smem) -> r
 
 }  // namespace
 
-size_t tv_workspace(const TVProblem& p) { return tv_layout(p).total; }
+size_t tv_workspace(const TVProblem& p) {
+  int NS, Lc;
+  tv_slices(p, nominal_resident(), NS, Lc);
+  return tv_layout(p, NS).total;
+}
 
-// Slices per row for this problem (the kernel needs W * NS resident CTAs).
+// The fewest slices per row this problem needs (the kernel needs W * NS
+// resident CTAs).
 int tv_slice_count(const TVProblem& p) {
   int NS, Lc;
-  tv_slices(p, NS, Lc);
+  tv_min_slices(p, NS, Lc);
   return NS;
 }
 
 cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_t* target_row,
                           const void* z_draft, float* a, float* prefix, float* loss, double* numer,
                           void* grad, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  const TVLayout L = tv_layout(p);
-  if (ws_bytes < L.total) return cudaErrorInvalidValue;
   if (p.W > kTVMaxW) return cudaErrorInvalidConfiguration;
   const int es = elt_size(p.logit_dtype);
   const int gs = elt_size(p.grad_dtype);
+  void* fn = pick_kernel(p.logit_dtype, p.grad_dtype);
+  // Resident CTAs at the budget's shared memory, the most any slice count
+  // uses: every CTA of the grid is then co-resident whatever NS is chosen.
+  const size_t smem_max = ((sizeof(TVShared) + 127) / 128) * 128 + (size_t)kTVSmemBudget;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int resident = 0;
+  cudaError_t e;
+  {
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    // The attribute is per function: set it on every launch (another problem
+    // size may have lowered it since).
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    auto key = std::make_tuple(dev, fn, (int)smem_max);
+    auto it = g_occ_cache.find(key);
+    if (it != g_occ_cache.end()) {
+      resident = it->second;
+    } else {
+      int per_sm = 0, nsm = 148;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kTVThreads, smem_max);
+      if (e != cudaSuccess) return e;
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+      resident = per_sm * nsm;
+      g_occ_cache[key] = resident;
+    }
+  }
   int NS, Lc;
-  tv_slices(p, NS, Lc);
+  tv_slices(p, resident, NS, Lc);
+  TVLayout L = tv_layout(p, NS);
+  if (ws_bytes < L.total) {  // sized for another device: the budget's slices
+    tv_min_slices(p, NS, Lc);
+    L = tv_layout(p, NS);
+  }
+  if (ws_bytes < L.total) return cudaErrorInvalidValue;
   if (NS > kTVMaxSlices) return cudaErrorInvalidConfiguration;
   const size_t smem = ((sizeof(TVShared) + 127) / 128) * 128 + 2ull * Lc * es;
 
@@ -636,34 +705,8 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
   A.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
   A.total_tasks = p.N * NS;
 
-  void* fn = pick_kernel(p.logit_dtype, p.grad_dtype);
-  cudaError_t e = cudaMemsetAsync(w + L.zero_begin, 0, L.zero_bytes, stream);
+  e = cudaMemsetAsync(w + L.zero_begin, 0, L.zero_bytes, stream);
   if (e != cudaSuccess) return e;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  int resident = 0;
-  {
-    std::lock_guard<std::mutex> lk(g_occ_mu);
-    // The attribute is per function: set it on every launch (another problem
-    // size may have lowered it since).
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               (int)cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    auto key = std::make_tuple(dev, fn, (int)smem);
-    auto it = g_occ_cache.find(key);
-    if (it != g_occ_cache.end()) {
-      resident = it->second;
-    } else {
-      int per_sm = 0, nsm = 148;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kTVThreads, smem);
-      if (e != cudaSuccess) return e;
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-      resident = per_sm * nsm;
-      g_occ_cache[key] = resident;
-    }
-  }
   // Every task of a branch must be able to be resident at once.  The grid is
   // a whole number of branches' worth of tasks when that idles under 5 % of
   // the resident slots, else every slot (see the kernel's schedule).
