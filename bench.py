@@ -242,8 +242,8 @@ def run_gpu(args):
     if st != 0:
         raise RuntimeError(f"device status {st:#x} after warm-up")
 
-    clk_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-    os.makedirs(os.path.dirname(clk_path), exist_ok=True)
+    import tempfile
+    clk_path = os.path.join(tempfile.gettempdir(), f"specopd_clocks_rank{rank}.csv")
     sampler, fh = _clock_sampler(clk_path) if rank == 0 else (None, None)
     time.sleep(0.3 if sampler else 0)
 
