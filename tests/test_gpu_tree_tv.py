@@ -233,7 +233,8 @@ def test_tv_8b_bf16_through_score_rows(lib):
     (111_104, 4, 2, "bf16", "f32"),  # ragged last slice, aligned path
     (40_000, 64, 2, "bf16", "f32"),  # W*NS = 256 tasks per branch, rounds of whole branches
     (151_936, 16, 3, "bf16", "f32"),  # the long trunk's vocabulary and W (NS = 12)
-    (248_320, 16, 4, "bf16", "f32"),  # the packed batch's vocabulary and W (NS = 37, one branch a round)
+    (248_320, 16, 4, "bf16", "f32"),  # the packed batch's vocabulary and W
+    (4096, 160, 1, "bf16", "f32"),   # W above the SM count: the slice schedule, aligned rows
 ])
 def test_tv_shapes(lib, V, W, nb, dtype, gdt):
     rng = np.random.default_rng(V + W)

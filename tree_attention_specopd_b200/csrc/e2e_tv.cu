@@ -536,6 +536,8 @@ __global__ void __launch_bounds__(kTVThreads, kTVCtasPerSm) e2e_tv_kernel(const 
   }
 }
 
+#include "e2e_tv_row.cuh"
+
 // ------------------------------------------------------------------ host
 namespace {
 
@@ -627,7 +629,7 @@ std::map<std::tuple<int, void*, int>, int> g_occ_cache;  // (dev, fn, smem) -> r
 size_t tv_workspace(const TVProblem& p) {
   int NS, Lc;
   tv_slices(p, nominal_resident(), NS, Lc);
-  return tv_layout(p, NS).total;
+  return std::max(tv_layout(p, NS).total, tvrow::row_layout(p).total);
 }
 
 // The fewest slices per row this problem needs (the kernel needs W * NS
@@ -638,12 +640,82 @@ int tv_slice_count(const TVProblem& p) {
   return NS;
 }
 
+namespace {
+
+template <typename Tin, typename Tg>
+void* row_kernel_ptr() {
+  return reinterpret_cast<void*>(&e2e_tv_row_kernel<Tin, Tg>);
+}
+
+void* pick_row_kernel(specopd_dtype in, specopd_dtype g) {
+  if (in == SPECOPD_BF16)
+    return g == SPECOPD_BF16 ? row_kernel_ptr<__nv_bfloat16, __nv_bfloat16>()
+                             : row_kernel_ptr<__nv_bfloat16, float>();
+  return g == SPECOPD_BF16 ? row_kernel_ptr<float, __nv_bfloat16>() : row_kernel_ptr<float, float>();
+}
+
+// Whole-row schedule (e2e_tv_row.cuh).  Returns cudaErrorNotSupported when
+// it does not apply (the slice schedule takes over).
+cudaError_t launch_row(const TVProblem& p, bool aligned, const void* z_target,
+                       const int32_t* target_row, const void* z_draft, float* a, float* prefix,
+                       float* loss, double* numer, void* grad, void* ws, size_t ws_bytes,
+                       cudaStream_t stream) {
+  using namespace tvrow;
+  if (!aligned) return cudaErrorNotSupported;
+  const tvrow::RowLayout L = row_layout(p);
+  if (ws_bytes < L.total) return cudaErrorNotSupported;
+  void* fn = pick_row_kernel(p.logit_dtype, p.grad_dtype);
+  const size_t smem = ((sizeof(tvrow::Shared) + 127) / 128) * 128 + (size_t)kStages * 2 * kChunkBytes;
+  int dev = 0, per_sm = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  // One CTA per SM keeps the rows in flight within the L2.
+  const long long resident = (long long)std::min(per_sm, 1) * nsm;
+  if (p.W > resident) return cudaErrorNotSupported;
+  const long long G = resident / p.W * p.W;  // whole branches per round
+  const int grid = (int)std::min<long long>(G, p.N);
+
+  RowArgs A;
+  A.nbranch = p.nbranch; A.W = p.W; A.V = p.V; A.N = p.N; A.rows_target = p.rows_target;
+  A.compute_grad = p.compute_grad && grad != nullptr;
+  A.norm = p.norm_count;
+  A.inv_norm = (float)(1.0 / p.norm_count);
+  A.zt = z_target; A.trow = target_row; A.zd = z_draft;
+  A.a_out = a; A.prefix = prefix; A.loss = loss; A.numer = numer; A.grad = grad;
+  char* w = reinterpret_cast<char*>(ws);
+  A.part = reinterpret_cast<float2*>(w + L.part);
+  A.bsum = reinterpret_cast<double*>(w + L.bsum);
+  A.br_cnt = reinterpret_cast<unsigned*>(w + L.br_cnt);
+  A.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
+  e = cudaMemsetAsync(w + L.zero_begin, 0, L.zero_bytes, stream);
+  if (e != cudaSuccess) return e;
+  void* args[] = {&A};
+  return cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, smem, stream);
+}
+
+}  // namespace
+
 cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_t* target_row,
                           const void* z_draft, float* a, float* prefix, float* loss, double* numer,
                           void* grad, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (p.W > kTVMaxW) return cudaErrorInvalidConfiguration;
   const int es = elt_size(p.logit_dtype);
   const int gs = elt_size(p.grad_dtype);
+  {
+    const bool cg = p.compute_grad && grad != nullptr;
+    const bool aligned = ((uintptr_t)z_target % 16 == 0) && ((uintptr_t)z_draft % 16 == 0) &&
+                         (!cg || (uintptr_t)grad % 16 == 0) && ((size_t)p.V * es % 16 == 0) &&
+                         (!cg || (size_t)p.V * gs % 16 == 0);
+    const cudaError_t e = launch_row(p, aligned, z_target, target_row, z_draft, a, prefix, loss,
+                                     numer, grad, ws, ws_bytes, stream);
+    if (e != cudaErrorNotSupported) return e;
+  }
   void* fn = pick_kernel(p.logit_dtype, p.grad_dtype);
   // Resident CTAs at the budget's shared memory, the most any slice count
   // uses: every CTA of the grid is then co-resident whatever NS is chosen.

@@ -7,26 +7,38 @@
 // touched, so no mask is materialised.
 //
 // This variant serves fp32 workloads (tiny problems where tensor cores do
-// not apply).  One CTA per (branch row, kv head); one warp per query head
-// of the GQA group; keys are visited in order with an online softmax, each
-// lane owning D/32 output dims.  q and branch k arrive already rotated.
+// not apply).  One CTA per (branch row, kv head); one warp per query head of
+// the GQA group.  Keys go in blocks of 32: lane l scores key kb + l with a
+// full dot product (q, pre-scaled, from shared memory), one warp reduction
+// gives the block's max, the running (max, sum, O) is rescaled once per
+// block, and P.V runs with the lanes over the output dims (the block's p
+// from shared memory).  q and branch k arrive already rotated.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace specopd {
 
-template <int DPL>  // dims per lane = D / 32
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+template <int D>
 __global__ void __launch_bounds__(1024) attn_simt_kernel(
     const AttnProblem p, const float* __restrict__ q_rot, const float* __restrict__ k_rot,
     const float* __restrict__ v_br, const float* __restrict__ k_tr,
     const float* __restrict__ v_tr, const int32_t* __restrict__ cu_trunk,
     const int32_t* __restrict__ anchors, float* __restrict__ out, float* __restrict__ lse) {
+  constexpr int DPL = D / 32;  // output dims per lane
+  extern __shared__ __align__(16) float simt_smem[];
   const int r = blockIdx.x;
   const int hk = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp >= p.G) return;
+  float* sq = simt_smem + warp * (D + 32);  // this head's scaled q
+  float* sp = sq + D;                       // p of the current key block
   const int h = hk * p.G + warp;
-  const int D = p.D;
   const int Wm1 = p.W - 1;
   const int bid = r / Wm1;
   const int i = r % Wm1 + 1;
@@ -41,38 +53,53 @@ __global__ void __launch_bounds__(1024) attn_simt_kernel(
     if (lse && lane == 0) lse[(long long)r * p.Hq + h] = __int_as_float(0x7fc00000);
     return;
   }
-  float q[DPL];
-  const float* qp = q_rot + ((long long)r * p.Hq + h) * D + lane * DPL;
-#pragma unroll
-  for (int d = 0; d < DPL; ++d) q[d] = qp[d] * p.scale;
+  const float* qp = q_rot + ((long long)r * p.Hq + h) * D;
+  for (int d = lane; d < D; d += 32) sq[d] = qp[d] * p.scale;
+  __syncwarp();
+  const int first = bid * Wm1;  // branch node (s,b,1) as a branch row index
+  const int nkeys = a + 1 + i;
+  auto key_row = [&](int kk) -> long long {
+    return kk <= a ? (long long)(t0 + kk) * p.Hkv + hk : (long long)(first + (kk - a - 1)) * p.Hkv + hk;
+  };
   float acc[DPL];
 #pragma unroll
   for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
   float m = -INFINITY, l = 0.f;
-  const int first = bid * Wm1;  // branch node (s,b,1) as a branch row index
-  const int nkeys = a + 1 + i;
-  for (int kk = 0; kk < nkeys; ++kk) {
-    const float* kp;
-    const float* vp;
-    if (kk <= a) {
-      const long long row = (long long)(t0 + kk) * p.Hkv + hk;
-      kp = k_tr + row * D;
-      vp = v_tr + row * D;
-    } else {
-      const long long row = (long long)(first + (kk - a - 1)) * p.Hkv + hk;
-      kp = k_rot + row * D;
-      vp = v_br + row * D;
+  for (int kb = 0; kb < nkeys; kb += 32) {
+    const int kk = kb + lane;
+    float sc = -INFINITY;
+    if (kk < nkeys) {
+      const float* kp = (kk <= a ? k_tr : k_rot) + key_row(kk) * D;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int d = 0; d < D; d += 8) {
+        const float4 k0 = *reinterpret_cast<const float4*>(kp + d);
+        const float4 k1 = *reinterpret_cast<const float4*>(kp + d + 4);
+        const float4 q0 = *reinterpret_cast<const float4*>(sq + d);
+        const float4 q1 = *reinterpret_cast<const float4*>(sq + d + 4);
+        s0 = fmaf(q0.x, k0.x, fmaf(q0.y, k0.y, fmaf(q0.z, k0.z, fmaf(q0.w, k0.w, s0))));
+        s1 = fmaf(q1.x, k1.x, fmaf(q1.y, k1.y, fmaf(q1.z, k1.z, fmaf(q1.w, k1.w, s1))));
+      }
+      sc = s0 + s1;
     }
-    float sdot = 0.f;
+    const float mn = fmaxf(m, warp_max_f(sc));
+    const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);  // first block: O and l are zero
+    const float pk = (kk < nkeys) ? expf(sc - mn) : 0.f;
+    l = l * corr + warp_sum(pk);
 #pragma unroll
-    for (int d = 0; d < DPL; ++d) sdot = fmaf(q[d], kp[lane * DPL + d], sdot);
-    sdot = warp_sum(sdot);
-    const float mn = fmaxf(m, sdot);
-    const float corr = expf(m - mn);  // m = -inf on the first key -> 0
-    const float pk = expf(sdot - mn);
-    l = l * corr + pk;
+    for (int d = 0; d < DPL; ++d) acc[d] *= corr;
+    sp[lane] = pk;
+    __syncwarp();
+    const int nb = min(32, nkeys - kb);
+#pragma unroll 8
+    for (int k = 0; k < nb; ++k) {
+      const int key = kb + k;
+      const float* vp = (key <= a ? v_tr : v_br) + key_row(key) * D + lane * DPL;
+      const float pkk = sp[k];
 #pragma unroll
-    for (int d = 0; d < DPL; ++d) acc[d] = fmaf(pk, vp[lane * DPL + d], acc[d] * corr);
+      for (int d = 0; d < DPL; ++d) acc[d] = fmaf(pkk, vp[d], acc[d]);
+    }
+    __syncwarp();  // sp is rewritten by the next block
     m = mn;
   }
   const float inv = 1.f / l;
@@ -86,14 +113,16 @@ cudaError_t launch_attn_simt_f32(const AttnProblem& p, const float* q_rot, const
                                  const int32_t* cu_trunk, const int32_t* anchors, float* out,
                                  float* lse, cudaStream_t st) {
   if (p.R == 0) return cudaSuccess;
+  if (p.G < 1 || p.G > 32) return cudaErrorInvalidValue;
   dim3 grid(p.R, p.Hkv);
   dim3 block(32 * p.G);
+  const size_t smem = (size_t)p.G * (p.D + 32) * sizeof(float);
   if (p.D == 64)
-    attn_simt_kernel<2><<<grid, block, 0, st>>>(p, q_rot, k_rot, v_br, k_tr, v_tr, cu_trunk,
-                                                anchors, out, lse);
+    attn_simt_kernel<64><<<grid, block, smem, st>>>(p, q_rot, k_rot, v_br, k_tr, v_tr, cu_trunk,
+                                                    anchors, out, lse);
   else if (p.D == 128)
-    attn_simt_kernel<4><<<grid, block, 0, st>>>(p, q_rot, k_rot, v_br, k_tr, v_tr, cu_trunk,
-                                                anchors, out, lse);
+    attn_simt_kernel<128><<<grid, block, smem, st>>>(p, q_rot, k_rot, v_br, k_tr, v_tr, cu_trunk,
+                                                     anchors, out, lse);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
