@@ -336,7 +336,11 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-TV_SOURCES = ("tree_attention_specopd_b200/csrc/e2e_tv.cu", "tree_attention_specopd_b200/csrc/common.cuh")
+TV_SOURCES = (
+    "tree_attention_specopd_b200/csrc/e2e_tv.cu",
+    "tree_attention_specopd_b200/csrc/e2e_tv_row.cuh",
+    "tree_attention_specopd_b200/csrc/common.cuh",
+)
 
 
 def tv_source_sha256():
