@@ -680,6 +680,10 @@ cudaError_t launch_row(const TVProblem& p, bool aligned, const void* z_target,
   if (p.W > resident) return cudaErrorNotSupported;
   const long long G = resident / p.W * p.W;  // whole branches per round
   const int grid = (int)std::min<long long>(G, p.N);
+  // The ring's chunk counter is 32-bit: keep a CTA's chunks below 2^32.
+  const long long ce = (long long)kConsumers * kVPT * (16 / elt_size(p.logit_dtype));
+  if ((long long)((p.N + G - 1) / G) * 3 * ((p.V + ce - 1) / ce) >= (1LL << 32))
+    return cudaErrorNotSupported;
 
   RowArgs A;
   A.nbranch = p.nbranch; A.W = p.W; A.V = p.V; A.N = p.N; A.rows_target = p.rows_target;

@@ -5,44 +5,55 @@
 // Same quantities as e2e_tv.cu (SpecOPD review (jaehun.me) §1.1, §3.3;
 // paper summary (rustineverything.app) §2.3).
 //
-// A CTA owns one supervised position n at a time and streams both logit
-// rows through a ring of shared-memory chunks three times:
+// A task is one supervised position n.  A CTA streams both logit rows of
+// its positions through a ring of shared-memory chunks, three passes per
+// position:
 //   A: the row statistics (maxima, sums of 2^(x - max)) -> lse of both rows
 //      (no other CTA is involved);
 //   B: the overlap a_n = sum_v min(p_v, q_v) and s_n = sum_{q<p} q_v;
 //      a_n and s_n are published for the branch;
 //   C: after the branch's W overlaps are in, the gradient row.
-// One producer warp issues the 1-D bulk copies (TMA) of every chunk of every
-// pass ahead of the consumers (24 warps); chunks of passes A and B are
-// fetched with an L2 evict-last hint, so passes B and C mostly re-read the
-// rows from L2, and pass C with evict-first.  The only cross-CTA wait is the
-// branch's, after pass B: the W positions of a branch are processed at the
-// same time by W CTAs.
+// The passes of consecutive tasks are pipelined: phase k interleaves pass A
+// of task k with pass C of task k - 1 chunk by chunk (A leads by kLag
+// chunks), then runs pass B of task k.  So each phase reads new rows from
+// DRAM while it writes the previous gradient row, the L2 holds about one
+// task's rows per CTA (pass C frees task k - 1's chunks as pass A brings in
+// task k's), and the branch handshake of task k - 1 has pass B of that task
+// and the first chunks of pass A of task k to complete in.
+//
+// Roles: one producer warp issues the 1-D bulk copies (TMA) of every chunk
+// ahead of the consumers (passes A and B with an L2 evict-last hint, pass C
+// with evict-first); 24 consumer warps do the arithmetic; one scorer warp
+// waits for each task's branch, computes g_n and the owner's outputs, and
+// hands g_n to the consumers through an mbarrier.
 //
 // Schedule: CTA g runs positions g, g + G, g + 2G, ... with G a multiple of
-// W and at most the resident CTAs, so every round holds whole branches and a
-// task waits only for tasks of its own round, each the current task of a
-// resident CTA: no deadlock.  One CTA per SM keeps the rows in flight
-// (G x 2 rows) within the L2.  Every wait is bounded.
+// W and at most the resident CTAs, so every round holds whole branches.  A
+// task's handshake waits only for the other positions of its branch, which
+// run on resident CTAs of the same round and publish after pass B, which
+// needs only earlier handshakes of the same CTAs: no deadlock.  One CTA per
+// SM keeps the rows in flight within the L2.  Every wait is bounded.
 
 namespace tvrow {
 
 constexpr int kConsumers = 768;              // 24 consumer warps
-constexpr int kThreads = kConsumers + 32;    // + the producer warp
 constexpr int kCWarps = kConsumers / 32;
+constexpr int kProducerWarp = kCWarps;       // issues the bulk copies
+constexpr int kScorerWarp = kCWarps + 1;     // branch handshake, g_n, owner outputs, loss
+constexpr int kThreads = kConsumers + 64;
 constexpr int kVPT = 2;                      // 16-byte vectors per consumer per row per chunk
 constexpr int kStages = 4;                   // ring depth (4 x 48 KB)
 constexpr int kChunkBytes = kConsumers * 16 * kVPT;  // bytes of one row per chunk
 constexpr int kMaxW = 256;
+constexpr int kLag = 4;                      // pass-A chunks ahead of pass C in a phase
 
 struct Shared {
   uint64_t full[kStages], empty[kStages];
-  float4 red[kCWarps];
-  double dred[kCWarps];
-  float2 lse;
-  float g, s_own;
-  int flag;
-  float sa[kMaxW];
+  uint64_t gfull;            // one phase per task: g_n and s_n are in
+  float4 red[2][kCWarps];    // per-warp (max, sum) of both rows after pass A, by task parity
+  float2 redB[kCWarps];      // per-warp (a, s) partials after pass B
+  float g, s_own;            // written by the scorer warp
+  float sa[kMaxW];           // the branch's overlaps (scorer warp)
 };
 
 // Row-task workspace: per-position (a, s) records, per-branch prefix-product
@@ -92,6 +103,9 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last_full() {
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+__device__ __forceinline__ void named_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 }  // namespace tvrow
 
@@ -109,7 +123,7 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
   const int nch = (V + CE - 1) / CE;   // chunks per row
   const int G = gridDim.x;
   const int ntask = (int)blockIdx.x < A.N ? (A.N - 1 - (int)blockIdx.x) / G + 1 : 0;
-  const int npass = A.compute_grad ? 3 : 2;
+  const bool grad = A.compute_grad != 0;
   const float2 L2E = make_float2(kLog2e, kLog2e);
   const float qnan = __int_as_float(0x7fc00000);
   auto target_row = [&](int n, bool& ok) -> int {
@@ -123,38 +137,120 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], kCWarps);
     }
+    mbar_init(&sh.gfull, 1);
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kCWarps) {
+  if (warp == kProducerWarp) {
     // ================================================================ producer
+    // Chunk order, shared with the consumers: for k = 0 .. ntask, phase k
+    // interleaves pass A of task k with pass C of task k - 1 (A leads by
+    // kLag chunks), then pass B of task k; phase ntask holds only the last C.
     if (lane == 0) {
       const uint64_t keep = l2_policy_evict_last_full();  // passes A, B: read again soon
       const uint64_t drop = l2_policy_evict_first();      // pass C: last use
       const Tin* zt = reinterpret_cast<const Tin*>(A.zt);
       const Tin* zd = reinterpret_cast<const Tin*>(A.zd);
-      long long q = 0;  // chunk sequence number over all tasks and passes
-      for (int k = 0; k < ntask; ++k) {
-        const int n = (int)blockIdx.x + k * G;
-        bool ok;
-        const Tin* rt = zt + (long long)target_row(n, ok) * V;
-        const Tin* rd = zd + (long long)n * V;
-        for (int pass = 0; pass < npass; ++pass) {
-          for (int c = 0; c < nch; ++c, ++q) {
-            const int st = (int)(q % kStages);
-            const long long use = q / kStages;
-            if (use > 0 && !mbar_wait(&sh.empty[st], (unsigned)((use - 1) & 1))) {
-              atomicExch(&A.ctl[2], 1u);
-              return;  // the consumers' waits run out in turn
-            }
-            const int e0 = c * CE;
-            const unsigned bytes = (unsigned)(min(CE, V - e0) * (int)sizeof(Tin));
-            uint8_t* dst = ring + (size_t)st * 2 * kChunkBytes;
-            mbar_arrive_expect_tx(&sh.full[st], 2u * bytes);
-            bulk_g2s_hint(dst, rt + e0, bytes, &sh.full[st], pass < 2 ? keep : drop);
-            bulk_g2s_hint(dst + kChunkBytes, rd + e0, bytes, &sh.full[st], pass < 2 ? keep : drop);
+      unsigned q = 0;  // chunk sequence number over all tasks and passes (mod 2^32)
+      bool live = true;
+      auto issue = [&](const Tin* rt, const Tin* rd, int c, uint64_t pol) {
+        if (!live) return;
+        const int st = (int)(q % kStages);
+        const unsigned use = q / kStages;
+        if (use > 0u && !mbar_wait(&sh.empty[st], (use - 1u) & 1u)) {
+          atomicExch(&A.ctl[2], 1u);
+          live = false;  // the consumers' waits run out in turn
+          return;
+        }
+        const int e0 = c * CE;
+        const unsigned bytes = (unsigned)(min(CE, V - e0) * (int)sizeof(Tin));
+        uint8_t* dst = ring + (size_t)st * 2 * kChunkBytes;
+        mbar_arrive_expect_tx(&sh.full[st], 2u * bytes);
+        bulk_g2s_hint(dst, rt + e0, bytes, &sh.full[st], pol);
+        bulk_g2s_hint(dst + kChunkBytes, rd + e0, bytes, &sh.full[st], pol);
+        ++q;
+      };
+      const Tin *rt_prev = zt, *rd_prev = zd;
+      for (int k = 0; k <= ntask && live; ++k) {
+        const bool hasA = k < ntask, hasC = grad && k > 0;
+        const Tin *rt = zt, *rd = zd;
+        if (hasA) {
+          const int n = (int)blockIdx.x + k * G;
+          bool ok;
+          rt = zt + (long long)target_row(n, ok) * V;
+          rd = zd + (long long)n * V;
+        }
+        for (int i = -kLag; i < nch; ++i) {
+          if (hasC && i >= 0) issue(rt_prev, rd_prev, i, drop);
+          if (hasA && i + kLag < nch) issue(rt, rd, i + kLag, keep);
+        }
+        if (hasA)
+          for (int c = 0; c < nch; ++c) issue(rt, rd, c, keep);
+        rt_prev = rt;
+        rd_prev = rd;
+      }
+    }
+    return;
+  }
+
+  if (warp == kScorerWarp) {
+    // ================================================================ scorer
+    // Per task, after the W positions of its branch have published (a, s):
+    // g_n for pass C, the owner's outputs, and the loss once every branch is
+    // in.  Runs beside the consumers, which need g_n only a few chunks into
+    // the next phase.
+    for (int k = 0; k < ntask; ++k) {
+      const int n = (int)blockIdx.x + k * G;
+      const int b = n / W, i = n % W;
+      const bool owner = (i == 0);  // writes the branch's overlaps and prefix products
+      int last = 0;
+      if (lane == 0) {
+        if (grad || owner) {
+          bool ok = __ldcg(&A.ctl[2]) == 0u;
+          if (ok) ok = wait_flag_geq(&A.br_cnt[b], (unsigned)W);
+          if (!ok) atomicExch(&A.ctl[2], 1u);
+          float s_own = qnan;
+          for (int j = 0; j < W; ++j) {
+            const float2 u = __ldcg(&A.part[(size_t)b * W + j]);
+            sh.sa[j] = ok ? u.x : qnan;
+            if (j == i) s_own = ok ? u.y : qnan;
           }
+          // g_n = -(1/norm) P_{i-1} S_i, with no division by any overlap
+          float P = 1.f;
+          for (int j = 0; j < i; ++j) P *= sh.sa[j];
+          float S = 1.f;
+          for (int j = W - 1; j > i; --j) S = fmaf(sh.sa[j], S, 1.f);
+          sh.g = -A.inv_norm * P * S;
+          sh.s_own = s_own;
+          if (owner) {
+            float Pp = 1.f;
+            double sumP = 0.0;
+            for (int j = 0; j < W; ++j) {
+              Pp *= sh.sa[j];
+              A.a_out[b * W + j] = sh.sa[j];
+              A.prefix[b * W + j] = Pp;
+              sumP += (double)Pp;
+            }
+            A.bsum[b] = sumP;
+            __threadfence();
+            if (atomicAdd(&A.ctl[1], 1u) == (unsigned)A.nbranch - 1u) {
+              __threadfence();
+              last = 1;
+            }
+          }
+        }
+        mbar_arrive(&sh.gfull);  // releases sh.g and sh.s_own to the consumers
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        // Last branch: loss = 1 - sum_b bsum[b] / norm, fixed summation order.
+        double acc = 0.0;
+        for (int j = lane; j < A.nbranch; j += 32) acc += __ldcg(&A.bsum[j]);
+        acc = warp_sum_d(acc);
+        if (lane == 0) {
+          A.loss[0] = (float)(1.0 - acc / A.norm);
+          if (A.numer) A.numer[0] = acc;
         }
       }
     }
@@ -162,14 +258,14 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
   }
 
   // ================================================================== consumers
-  long long q = 0;
+  unsigned q = 0;
   bool dead = false;  // a wait ran out: skip the remaining waits
   // Wait for chunk q, return its two row vectors of this thread (valid when
   // the element index is below V).
   // Vector v of this thread in chunk c: elements c*CE + (v*kConsumers + tid)*VN.
   auto wait_chunk = [&]() {
     const int st = (int)(q % kStages);
-    if (!dead && !mbar_wait(&sh.full[st], (unsigned)((q / kStages) & 1))) {
+    if (!dead && !mbar_wait(&sh.full[st], (q / kStages) & 1u)) {
       dead = true;
       atomicExch(&A.ctl[2], 1u);
     }
@@ -192,85 +288,147 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
     ++q;
   };
 
-  for (int k = 0; k < ntask; ++k) {
-    const int n = (int)blockIdx.x + k * G;
-    const int b = n / W, i = n % W;
+  // lse (log2 units) of the position whose gradient the next phase writes
+  float lseC_t = 0.f, lseC_d = 0.f;
+  for (int k = 0; k <= ntask; ++k) {
+    const bool hasA = k < ntask, hasC = grad && k > 0;
+    const int n = (int)blockIdx.x + k * G;  // task k (pass A, B); n - G is task k - 1
 
-    // ---------------------------------------------- pass A: row statistics
-    float mt = -INFINITY, md = -INFINITY, sum_t, sum_d;
-    {
-      float2 at0 = make_float2(0.f, 0.f), at1 = at0, ad0 = at0, ad1 = at0;
-      auto raise = [](float gm, float& m, float2& s0, float2& s1) {
-        if (gm > m) {
-          const float f = (m == -INFINITY) ? 0.f : ex2_fast(m - gm);
-          s0 = (m == -INFINITY) ? make_float2(0.f, 0.f) : __fmul2_rn(s0, make_float2(f, f));
-          s1 = (m == -INFINITY) ? make_float2(0.f, 0.f) : __fmul2_rn(s1, make_float2(f, f));
-          m = gm;
+    // ------------------------------ phase k: pass A of task k, pass C of task k - 1
+    float mt = -INFINITY, md = -INFINITY;
+    float2 at0 = make_float2(0.f, 0.f), at1 = at0, ad0 = at0, ad1 = at0;
+    auto raise = [](float gm, float& m, float2& s0, float2& s1) {
+      if (gm > m) {
+        const float f = (m == -INFINITY) ? 0.f : ex2_fast(m - gm);
+        s0 = (m == -INFINITY) ? make_float2(0.f, 0.f) : __fmul2_rn(s0, make_float2(f, f));
+        s1 = (m == -INFINITY) ? make_float2(0.f, 0.f) : __fmul2_rn(s1, make_float2(f, f));
+        m = gm;
+      }
+    };
+    const float2 nLtC = make_float2(-lseC_t, -lseC_t), nLdC = make_float2(-lseC_d, -lseC_d);
+    float c1 = 0.f, c0 = 0.f;  // gradient coefficient for [q<p] = 1 / 0
+    Tg* gout = reinterpret_cast<Tg*>(A.grad) + (hasC ? (long long)(n - G) * V : 0LL);
+    for (int i = -kLag; i < nch; ++i) {
+      if (hasC && i >= 0) {
+        // ---- pass C, chunk i: the gradient row of task k - 1
+        if (i == 0) {
+          if (!dead && !mbar_wait(&sh.gfull, (unsigned)((k - 1) & 1))) {
+            dead = true;
+            atomicExch(&A.ctl[2], 1u);
+          }
+          const float g = sh.g, s_val = sh.s_own;
+          c1 = g * (1.f - s_val);
+          c0 = -g * s_val;
         }
-      };
-      for (int c = 0; c < nch; ++c) {
         wait_chunk();
 #pragma unroll
         for (int v = 0; v < kVPT; ++v) {
-        uint4 ut, ud;
-        if (take(c, v, ut, ud)) {
-          raise(Vec<Tin>::vmax(ut) * kLog2e, mt, at0, at1);
-          raise(Vec<Tin>::vmax(ud) * kLog2e, md, ad0, ad1);
-          float2 ft[VP], fd[VP];
-          Vec<Tin>::pairs(ut, ft);
-          Vec<Tin>::pairs(ud, fd);
-          const float2 nmt = make_float2(-mt, -mt), nmd = make_float2(-md, -md);
+          uint4 ut, ud;
+          if (take(i, v, ut, ud)) {
+            float2 ft[VP], fd[VP], o[VP];
+            Vec<Tin>::pairs(ut, ft);
+            Vec<Tin>::pairs(ud, fd);
 #pragma unroll
-          for (int p = 0; p < VP; p += 2) {
-            at0 = __fadd2_rn(at0, ex2_pair(__ffma2_rn(ft[p], L2E, nmt)));
-            ad0 = __fadd2_rn(ad0, ex2_pair(__ffma2_rn(fd[p], L2E, nmd)));
-            at1 = __fadd2_rn(at1, ex2_pair(__ffma2_rn(ft[p + 1], L2E, nmt)));
-            ad1 = __fadd2_rn(ad1, ex2_pair(__ffma2_rn(fd[p + 1], L2E, nmd)));
+            for (int p = 0; p < VP; ++p) {
+              const float2 lt = __ffma2_rn(ft[p], L2E, nLtC);
+              const float2 ld = __ffma2_rn(fd[p], L2E, nLdC);
+              const float2 coef = make_float2(ld.x < lt.x ? c1 : c0, ld.y < lt.y ? c1 : c0);
+              o[p] = __fmul2_rn(ex2_pair(ld), coef);
+            }
+            Tg* dst = gout + i * CE + (v * kConsumers + tid) * VN;
+            if constexpr (sizeof(Tg) == 4) {
+#pragma unroll
+              for (int p = 0; p < VP; p += 2)
+                __stcs(reinterpret_cast<float4*>(dst + 2 * p),
+                       make_float4(o[p].x, o[p].y, o[p + 1].x, o[p + 1].y));
+            } else if constexpr (VP == 4) {
+              uint4 u;
+              u.x = pack_bf16x2(o[0].x, o[0].y);
+              u.y = pack_bf16x2(o[1].x, o[1].y);
+              u.z = pack_bf16x2(o[2].x, o[2].y);
+              u.w = pack_bf16x2(o[3].x, o[3].y);
+              __stcs(reinterpret_cast<uint4*>(dst), u);
+            } else {
+              uint2 u;
+              u.x = pack_bf16x2(o[0].x, o[0].y);
+              u.y = pack_bf16x2(o[1].x, o[1].y);
+              __stcs(reinterpret_cast<uint2*>(dst), u);
+            }
           }
-        }
         }
         give();
       }
-      sum_t = (at0.x + at0.y) + (at1.x + at1.y);
-      sum_d = (ad0.x + ad0.y) + (ad1.x + ad1.y);
-      // -inf maximum: this thread saw no finite entry of that row, no mass
-      if (mt == -INFINITY) sum_t = 0.f;
-      if (md == -INFINITY) sum_d = 0.f;
-    }
-    warp_lse2(mt, sum_t);
-    warp_lse2(md, sum_d);
-    if (lane == 0) sh.red[warp] = make_float4(mt, sum_t, md, sum_d);
-    named_sync(1, kConsumers);
-    if (tid == 0) {
-      float4 v = sh.red[0];
-      for (int w = 1; w < kCWarps; ++w) {
-        lse2_combine(v.x, v.y, sh.red[w].x, sh.red[w].y);
-        lse2_combine(v.z, v.w, sh.red[w].z, sh.red[w].w);
-      }
-      float2 L = make_float2(v.x + log2f(v.y), v.z + log2f(v.w));
-      bool row_ok;
-      target_row(n, row_ok);
-      if (!row_ok) {
-        set_status(SPECOPD_DEV_ROW_RANGE);
-        L = make_float2(qnan, qnan);
-      } else if (v.x == -INFINITY || v.z == -INFINITY) {
-        set_status(SPECOPD_DEV_ALL_NEG_INF);
-        L = make_float2(qnan, qnan);
-      }
-      if (dead) L = make_float2(qnan, qnan);
-      sh.lse = L;
-    }
-    named_sync(1, kConsumers);
-    const float lse2_t = sh.lse.x, lse2_d = sh.lse.y;
-    const float2 nLt = make_float2(-lse2_t, -lse2_t), nLd = make_float2(-lse2_d, -lse2_d);
-
-    // ---------------------------------------------- pass B: a_n and s_n
-    {
-      float2 pa2 = make_float2(0.f, 0.f), ps2 = pa2;
-      for (int c = 0; c < nch; ++c) {
+      if (hasA && i + kLag < nch) {
+        // ---- pass A, chunk i + kLag: row maxima and sums under a running maximum
+        const int c = i + kLag;
         wait_chunk();
 #pragma unroll
         for (int v = 0; v < kVPT; ++v) {
+          uint4 ut, ud;
+          if (take(c, v, ut, ud)) {
+            raise(Vec<Tin>::vmax(ut) * kLog2e, mt, at0, at1);
+            raise(Vec<Tin>::vmax(ud) * kLog2e, md, ad0, ad1);
+            float2 ft[VP], fd[VP];
+            Vec<Tin>::pairs(ut, ft);
+            Vec<Tin>::pairs(ud, fd);
+            const float2 nmt = make_float2(-mt, -mt), nmd = make_float2(-md, -md);
+#pragma unroll
+            for (int p = 0; p < VP; p += 2) {
+              at0 = __fadd2_rn(at0, ex2_pair(__ffma2_rn(ft[p], L2E, nmt)));
+              ad0 = __fadd2_rn(ad0, ex2_pair(__ffma2_rn(fd[p], L2E, nmd)));
+              at1 = __fadd2_rn(at1, ex2_pair(__ffma2_rn(ft[p + 1], L2E, nmt)));
+              ad1 = __fadd2_rn(ad1, ex2_pair(__ffma2_rn(fd[p + 1], L2E, nmd)));
+            }
+          }
+        }
+        give();
+      }
+    }
+    if (!hasA) break;  // the last phase held only the last gradient row
+    const int b = n / W;
+
+    // ------------------------------ lse of task k
+    float sum_t = (at0.x + at0.y) + (at1.x + at1.y);
+    float sum_d = (ad0.x + ad0.y) + (ad1.x + ad1.y);
+    // -inf maximum: this thread saw no finite entry of that row, no mass
+    if (mt == -INFINITY) sum_t = 0.f;
+    if (md == -INFINITY) sum_d = 0.f;
+    warp_lse2(mt, sum_t);
+    warp_lse2(md, sum_d);
+    if (lane == 0) sh.red[k & 1][warp] = make_float4(mt, sum_t, md, sum_d);
+    named_sync(1, kConsumers);
+    // Every warp combines the warp records itself (no second barrier).  The
+    // combination is symmetric in its two operands, so the butterfly leaves
+    // the same bits in every lane, and every warp computes the same L.  The
+    // records alternate between two buffers by task parity: a warp reaches
+    // the next write of this buffer only through the next task's barrier.
+    float2 L;
+    {
+      float4 v = lane < kCWarps ? sh.red[k & 1][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+      warp_lse2(v.x, v.y);
+      warp_lse2(v.z, v.w);
+      L = make_float2(v.x + log2f(v.y), v.z + log2f(v.w));
+      bool row_ok;
+      target_row(n, row_ok);
+      if (!row_ok) {
+        if (tid == 0) set_status(SPECOPD_DEV_ROW_RANGE);
+        L = make_float2(qnan, qnan);
+      } else if (v.x == -INFINITY || v.z == -INFINITY) {
+        if (tid == 0) set_status(SPECOPD_DEV_ALL_NEG_INF);
+        L = make_float2(qnan, qnan);
+      }
+      if (dead) L = make_float2(qnan, qnan);
+    }
+    lseC_t = L.x;
+    lseC_d = L.y;
+    const float2 nLt = make_float2(-L.x, -L.x), nLd = make_float2(-L.y, -L.y);
+
+    // ------------------------------ pass B of task k: a_n and s_n
+    float2 pa2 = make_float2(0.f, 0.f), ps2 = pa2;
+    for (int c = 0; c < nch; ++c) {
+      wait_chunk();
+#pragma unroll
+      for (int v = 0; v < kVPT; ++v) {
         uint4 ut, ud;
         if (take(c, v, ut, ud)) {
           float2 ft[VP], fd[VP];
@@ -285,123 +443,30 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
             ps2 = __fadd2_rn(ps2, make_float2(ld.x < lt.x ? e.x : 0.f, ld.y < lt.y ? e.y : 0.f));
           }
         }
-        }
-        give();
       }
+      give();
+    }
+    {
       const float pa = warp_sum(pa2.x + pa2.y);
       const float ps = warp_sum(ps2.x + ps2.y);
-      if (lane == 0) sh.red[warp] = make_float4(pa, ps, 0.f, 0.f);
+      if (lane == 0) sh.redB[warp] = make_float2(pa, ps);
     }
-    named_sync(1, kConsumers);
-    const bool owner = (i == 0);  // writes the branch's overlaps and prefix products
-    const bool need_branch = A.compute_grad || owner;
-    if (tid == 0) {
-      float2 v = make_float2(0.f, 0.f);
-      for (int w = 0; w < kCWarps; ++w) {
-        v.x += sh.red[w].x;
-        v.y += sh.red[w].y;
-      }
-      A.part[n] = v;
-      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&A.br_cnt[b]) : "memory");
-      int last = 0;
-      if (need_branch) {
-        // The W positions of the branch run in this round on W CTAs.
-        bool ok = !dead && __ldcg(&A.ctl[2]) == 0u;
-        if (ok) ok = wait_flag_geq(&A.br_cnt[b], (unsigned)W);
-        if (!ok) atomicExch(&A.ctl[2], 1u);
-        for (int j = 0; j < W; ++j) {
-          const float2 u = __ldcg(&A.part[(size_t)b * W + j]);
-          sh.sa[j] = ok ? u.x : qnan;
-          if (j == i) sh.s_own = ok ? u.y : qnan;
-        }
-        // g_n = -(1/norm) P_{i-1} S_i, with no division by any overlap
-        float P = 1.f;
-        for (int j = 0; j < i; ++j) P *= sh.sa[j];
-        float S = 1.f;
-        for (int j = W - 1; j > i; --j) S = fmaf(sh.sa[j], S, 1.f);
-        sh.g = -A.inv_norm * P * S;
-        if (owner) {
-          float Pp = 1.f;
-          double sumP = 0.0;
-          for (int j = 0; j < W; ++j) {
-            Pp *= sh.sa[j];
-            A.a_out[b * W + j] = sh.sa[j];
-            A.prefix[b * W + j] = Pp;
-            sumP += (double)Pp;
-          }
-          A.bsum[b] = sumP;
-          __threadfence();
-          if (atomicAdd(&A.ctl[1], 1u) == (unsigned)A.nbranch - 1u) {
-            __threadfence();
-            last = 1;
-          }
-        }
-      }
-      sh.flag = last;
-    }
-    named_sync(1, kConsumers);
-    if (sh.flag) {
-      // Last branch: loss = 1 - sum_b bsum[b] / norm, fixed summation order.
-      double acc = 0.0;
-      for (int j = tid; j < A.nbranch; j += kConsumers) acc += __ldcg(&A.bsum[j]);
-      acc = warp_sum_d(acc);
-      if (lane == 0) sh.dred[warp] = acc;
-      named_sync(1, kConsumers);
+    // Warp 0 collects the partials and publishes (a_n, s_n); the other warps
+    // go on to the next phase.  sh.redB is written again only after the next
+    // task's lse barrier, which warp 0 reaches after reading it.
+    if (warp == 0) {
+      named_sync(2, kConsumers);
       if (tid == 0) {
-        double tot = 0.0;
-        for (int w = 0; w < kCWarps; ++w) tot += sh.dred[w];
-        A.loss[0] = (float)(1.0 - tot / A.norm);
-        if (A.numer) A.numer[0] = tot;
-      }
-    }
-
-    // ---------------------------------------------- pass C: gradient row
-    if (A.compute_grad) {
-      const float g = sh.g, s_val = sh.s_own;
-      const float c1 = g * (1.f - s_val), c0 = -g * s_val;  // coefficient for [q<p] = 1 / 0
-      Tg* gout = reinterpret_cast<Tg*>(A.grad) + (long long)n * V;
-      for (int c = 0; c < nch; ++c) {
-        wait_chunk();
-#pragma unroll
-        for (int v = 0; v < kVPT; ++v) {
-        uint4 ut, ud;
-        if (take(c, v, ut, ud)) {
-          float2 ft[VP], fd[VP], o[VP];
-          Vec<Tin>::pairs(ut, ft);
-          Vec<Tin>::pairs(ud, fd);
-#pragma unroll
-          for (int p = 0; p < VP; ++p) {
-            const float2 lt = __ffma2_rn(ft[p], L2E, nLt);
-            const float2 ld = __ffma2_rn(fd[p], L2E, nLd);
-            const float2 coef = make_float2(ld.x < lt.x ? c1 : c0, ld.y < lt.y ? c1 : c0);
-            o[p] = __fmul2_rn(ex2_pair(ld), coef);
-          }
-          Tg* dst = gout + c * CE + (v * kConsumers + tid) * VN;
-          if constexpr (sizeof(Tg) == 4) {
-#pragma unroll
-            for (int p = 0; p < VP; p += 2)
-              __stcs(reinterpret_cast<float4*>(dst + 2 * p),
-                     make_float4(o[p].x, o[p].y, o[p + 1].x, o[p + 1].y));
-          } else if constexpr (VP == 4) {
-            uint4 u;
-            u.x = pack_bf16x2(o[0].x, o[0].y);
-            u.y = pack_bf16x2(o[1].x, o[1].y);
-            u.z = pack_bf16x2(o[2].x, o[2].y);
-            u.w = pack_bf16x2(o[3].x, o[3].y);
-            __stcs(reinterpret_cast<uint4*>(dst), u);
-          } else {
-            uint2 u;
-            u.x = pack_bf16x2(o[0].x, o[0].y);
-            u.y = pack_bf16x2(o[1].x, o[1].y);
-            __stcs(reinterpret_cast<uint2*>(dst), u);
-          }
+        float2 v = make_float2(0.f, 0.f);
+        for (int w = 0; w < kCWarps; ++w) {
+          v.x += sh.redB[w].x;
+          v.y += sh.redB[w].y;
         }
-        }
-        give();
+        A.part[n] = v;
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&A.br_cnt[b]) : "memory");
       }
+    } else {
+      named_arrive(2, kConsumers);
     }
-    // sh.lse, sh.g, sh.s_own and sh.red are rewritten by the next task only
-    // after its pass A, which every consumer reaches past this point.
-    named_sync(1, kConsumers);
   }
 }
