@@ -305,6 +305,25 @@ def test_tv_norm_count_and_no_grad(lib):
     assert abs(r2["loss"].item() - full["loss"]) < 1e-5
 
 
+def test_tv_no_grad_many_tasks(lib):
+    # Many positions per CTA without the gradient: the overlaps, prefix
+    # products and loss are the same bits as with it, and match the oracle.
+    rng = np.random.default_rng(11)
+    nb, W, V = 512, 4, 2000
+    zt = (2.0 * rng.standard_normal((nb * W, V))).astype(np.float32)
+    zd = (zt + rng.standard_normal((nb * W, V))).astype(np.float32)
+    zt = torch.from_numpy(zt).to(torch.bfloat16).float().numpy()
+    zd = torch.from_numpy(zd).to(torch.bfloat16).float().numpy()
+    ref = otv.e2e_tv(zt, None, zd, nb, W, compute_grad=False)
+    rg = _tv_run(lib, zt, zd, nb, W, "bf16", compute_grad=True)
+    rn = _tv_run(lib, zt, zd, nb, W, "bf16", compute_grad=False)
+    assert rn["grad"] is None
+    for k in ("a", "prefix", "loss", "numer"):
+        assert torch.equal(rg[k], rn[k]), k
+    assert rel_err(to_np(rn["a"]), ref["a"]) < 1e-5
+    assert abs(rn["loss"].item() - ref["loss"]) <= 1e-4 * abs(ref["loss"]) + 1e-7
+
+
 def test_tv_deterministic(lib):
     cfg = synth.tv_config("tiny")
     zt, zd = synth.logits(cfg)

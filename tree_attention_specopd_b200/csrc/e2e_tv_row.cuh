@@ -24,8 +24,9 @@
 // Roles: one producer warp issues the 1-D bulk copies (TMA) of every chunk
 // ahead of the consumers (passes A and B with an L2 evict-last hint, pass C
 // with evict-first); 24 consumer warps do the arithmetic; one scorer warp
-// waits for each task's branch, computes g_n and the owner's outputs, and
-// hands g_n to the consumers through an mbarrier.
+// publishes each task's (a_n, s_n) from the consumer warps' partials, waits
+// for the branch, computes g_n and the owner's outputs, and hands g_n to the
+// consumers through an mbarrier.
 //
 // Schedule: CTA g runs positions g, g + G, g + 2G, ... with G a multiple of
 // W and at most the resident CTAs, so every round holds whole branches.  A
@@ -49,6 +50,7 @@ constexpr int kLag = 4;                      // pass-A chunks ahead of pass C in
 
 struct Shared {
   uint64_t full[kStages], empty[kStages];
+  uint64_t bdone;            // one phase per task: every consumer warp's pass-B partials are in
   uint64_t gfull;            // one phase per task: g_n and s_n are in
   float4 red[2][kCWarps];    // per-warp (max, sum) of both rows after pass A, by task parity
   float2 redB[kCWarps];      // per-warp (a, s) partials after pass B
@@ -103,8 +105,23 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last_full() {
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-__device__ __forceinline__ void named_arrive(int id, int n) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+// (max, sum) pair of log2-domain statistics: combine two, branch-free.  An
+// empty side (max = -inf) contributes nothing; the result is symmetric in
+// the two operands bit for bit.
+__device__ __forceinline__ void lse2_merge(float& m, float& s, float m2, float s2) {
+  const float mn = fmaxf(m, m2);
+  const float a = (m == -INFINITY) ? 0.f : s * ex2_fast(m - mn);
+  const float b = (m2 == -INFINITY) ? 0.f : s2 * ex2_fast(m2 - mn);
+  m = mn;
+  s = a + b;
+}
+__device__ __forceinline__ void warp_lse2_merge(float& m, float& s) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    lse2_merge(m, s, m2, s2);
+  }
 }
 
 }  // namespace tvrow
@@ -137,6 +154,7 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], kCWarps);
     }
+    mbar_init(&sh.bdone, kCWarps);
     mbar_init(&sh.gfull, 1);
     fence_mbar_init();
   }
@@ -206,8 +224,22 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       const bool owner = (i == 0);  // writes the branch's overlaps and prefix products
       int last = 0;
       if (lane == 0) {
+        // publish (a_n, s_n) once the 24 consumer warps' partials are in
+        bool in = mbar_wait(&sh.bdone, (unsigned)(k & 1));
+        float2 v = make_float2(qnan, qnan);
+        if (in) {
+          v = make_float2(0.f, 0.f);
+          for (int w = 0; w < kCWarps; ++w) {
+            v.x += sh.redB[w].x;
+            v.y += sh.redB[w].y;
+          }
+        } else {
+          atomicExch(&A.ctl[2], 1u);
+        }
+        A.part[n] = v;
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&A.br_cnt[b]) : "memory");
         if (grad || owner) {
-          bool ok = __ldcg(&A.ctl[2]) == 0u;
+          bool ok = in && __ldcg(&A.ctl[2]) == 0u;
           if (ok) ok = wait_flag_geq(&A.br_cnt[b], (unsigned)W);
           if (!ok) atomicExch(&A.ctl[2], 1u);
           float s_own = qnan;
@@ -308,6 +340,12 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
     const float2 nLtC = make_float2(-lseC_t, -lseC_t), nLdC = make_float2(-lseC_d, -lseC_d);
     float c1 = 0.f, c0 = 0.f;  // gradient coefficient for [q<p] = 1 / 0
     Tg* gout = reinterpret_cast<Tg*>(A.grad) + (hasC ? (long long)(n - G) * V : 0LL);
+    if (!grad && k > 0 && !dead && !mbar_wait(&sh.gfull, (unsigned)((k - 1) & 1))) {
+      // Without pass C the consumers still keep within one task of the
+      // scorer, which reads sh.redB of the previous task.
+      dead = true;
+      atomicExch(&A.ctl[2], 1u);
+    }
     for (int i = -kLag; i < nch; ++i) {
       if (hasC && i >= 0) {
         // ---- pass C, chunk i: the gradient row of task k - 1
@@ -385,7 +423,6 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       }
     }
     if (!hasA) break;  // the last phase held only the last gradient row
-    const int b = n / W;
 
     // ------------------------------ lse of task k
     float sum_t = (at0.x + at0.y) + (at1.x + at1.y);
@@ -393,8 +430,8 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
     // -inf maximum: this thread saw no finite entry of that row, no mass
     if (mt == -INFINITY) sum_t = 0.f;
     if (md == -INFINITY) sum_d = 0.f;
-    warp_lse2(mt, sum_t);
-    warp_lse2(md, sum_d);
+    warp_lse2_merge(mt, sum_t);
+    warp_lse2_merge(md, sum_d);
     if (lane == 0) sh.red[k & 1][warp] = make_float4(mt, sum_t, md, sum_d);
     named_sync(1, kConsumers);
     // Every warp combines the warp records itself (no second barrier).  The
@@ -405,8 +442,8 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
     float2 L;
     {
       float4 v = lane < kCWarps ? sh.red[k & 1][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-      warp_lse2(v.x, v.y);
-      warp_lse2(v.z, v.w);
+      warp_lse2_merge(v.x, v.y);
+      warp_lse2_merge(v.z, v.w);
       L = make_float2(v.x + log2f(v.y), v.z + log2f(v.w));
       bool row_ok;
       target_row(n, row_ok);
@@ -446,27 +483,16 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       }
       give();
     }
+    // Partials to the scorer warp, which publishes them; no consumer waits.
+    // sh.redB is written again only after the scorer's gfull arrival for
+    // this task, which follows its read of sh.redB.
     {
       const float pa = warp_sum(pa2.x + pa2.y);
       const float ps = warp_sum(ps2.x + ps2.y);
-      if (lane == 0) sh.redB[warp] = make_float2(pa, ps);
-    }
-    // Warp 0 collects the partials and publishes (a_n, s_n); the other warps
-    // go on to the next phase.  sh.redB is written again only after the next
-    // task's lse barrier, which warp 0 reaches after reading it.
-    if (warp == 0) {
-      named_sync(2, kConsumers);
-      if (tid == 0) {
-        float2 v = make_float2(0.f, 0.f);
-        for (int w = 0; w < kCWarps; ++w) {
-          v.x += sh.redB[w].x;
-          v.y += sh.redB[w].y;
-        }
-        A.part[n] = v;
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&A.br_cnt[b]) : "memory");
+      if (lane == 0) {
+        sh.redB[warp] = make_float2(pa, ps);
+        mbar_arrive(&sh.bdone);
       }
-    } else {
-      named_arrive(2, kConsumers);
     }
   }
 }
