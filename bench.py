@@ -287,7 +287,7 @@ def run_gpu(args):
         tv_gbs = pb.tv_bytes / (tv_ms / 1e3) / 1e9
         attn_tflops = pb.flops / (attn_ms / 1e3) / 1e12
         clocks = _clock_summary(clk_path, local)
-        traffic = _ncu_traffic()
+        traffic = _ncu_traffic() if wl == WORKLOAD else None  # counters of the 8B launch
         line = {
             "metric": METRIC,
             "value": value,
@@ -354,8 +354,9 @@ def tv_source_sha256():
 
 
 def _ncu_traffic():
-    """DRAM bytes per e2e_tv launch from the committed ncu summary, or None
-    when it is absent or was taken on other kernel sources."""
+    """DRAM bytes per e2e_tv launch of the 8B-shaped workload from the
+    committed ncu summary, or None when it is absent or was taken on other
+    kernel sources."""
     path = os.path.join(ROOT, "profiles", "e2e_tv_8b_traffic.json")
     try:
         rec = json.load(open(path))
