@@ -277,6 +277,33 @@ def test_tv_special_rows(lib):
     assert _status(lib) == 0
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_tv_row_maxima_across_chunks(lib, dtype):
+    # Rows long enough for several shared-memory chunks, whose maxima appear
+    # late: a first stretch 100 nats below the rest (longer than a chunk),
+    # a leading run of -inf longer than a chunk, slowly and quickly rising
+    # rows.
+    V = 40_000
+    rng = np.random.default_rng(17)
+    zt = (2.0 * rng.standard_normal((8, V))).astype(np.float32)
+    zd = (zt + rng.standard_normal((8, V))).astype(np.float32)
+    zt[1, :15_000] -= 100.0
+    zd[1, :15_000] -= 100.0
+    zt[2, :20_000] = -np.inf
+    zd[3, :13_000] = -np.inf
+    zt[3, :15_000] -= 100.0
+    zt[4] = np.linspace(-50.0, 50.0, V)
+    zd[4] = zt[4] + rng.standard_normal(V).astype(np.float32)
+    zd[5] = np.linspace(-200.0, 200.0, V)
+    if dtype == "bf16":
+        zt = synth.round_bf16(zt)
+        zd = synth.round_bf16(zd)
+    ref = otv.e2e_tv(zt, None, zd, 2, 4)
+    res = _tv_run(lib, zt, zd, 2, 4, dtype)
+    _check_tv(res, ref)
+    assert _status(lib) == 0
+
+
 def test_tv_all_neg_inf_row_flags(lib):
     zt = np.zeros((2, 16), np.float32)
     zd = np.zeros((2, 16), np.float32)

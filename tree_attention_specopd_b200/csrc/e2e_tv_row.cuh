@@ -407,25 +407,66 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
         give();
       }
       if (hasA && i + kLag < nch) {
-        // ---- pass A, chunk i + kLag: row maxima and sums under a running maximum
+        // ---- pass A, chunk i + kLag: row sums under a running maximum.
+        // From the second chunk on, the chunk is summed under the current
+        // maxima first and accepted when both partial sums stay at most
+        // 2^64 (no term overflowed, none was -inf - -inf); otherwise, and
+        // for the first chunk, every vector raises the maxima before it is
+        // summed.  Either way the sums are of 2^(x - m) for the m they are
+        // kept under, so the lse below is the same quantity.
         const int c = i + kLag;
         wait_chunk();
+        uint4 ut[kVPT], ud[kVPT];
+        bool in[kVPT];
 #pragma unroll
-        for (int v = 0; v < kVPT; ++v) {
-          uint4 ut, ud;
-          if (take(c, v, ut, ud)) {
-            raise(Vec<Tin>::vmax(ut) * kLog2e, mt, at0, at1);
-            raise(Vec<Tin>::vmax(ud) * kLog2e, md, ad0, ad1);
-            float2 ft[VP], fd[VP];
-            Vec<Tin>::pairs(ut, ft);
-            Vec<Tin>::pairs(ud, fd);
-            const float2 nmt = make_float2(-mt, -mt), nmd = make_float2(-md, -md);
+        for (int v = 0; v < kVPT; ++v) in[v] = take(c, v, ut[v], ud[v]);
+        bool exact = (c == 0);
+        if (!exact) {
+          float2 ct0 = make_float2(0.f, 0.f), ct1 = ct0, cd0 = ct0, cd1 = ct0;
+          const float2 nmt = make_float2(-mt, -mt), nmd = make_float2(-md, -md);
 #pragma unroll
-            for (int p = 0; p < VP; p += 2) {
-              at0 = __fadd2_rn(at0, ex2_pair(__ffma2_rn(ft[p], L2E, nmt)));
-              ad0 = __fadd2_rn(ad0, ex2_pair(__ffma2_rn(fd[p], L2E, nmd)));
-              at1 = __fadd2_rn(at1, ex2_pair(__ffma2_rn(ft[p + 1], L2E, nmt)));
-              ad1 = __fadd2_rn(ad1, ex2_pair(__ffma2_rn(fd[p + 1], L2E, nmd)));
+          for (int v = 0; v < kVPT; ++v) {
+            if (in[v]) {
+              float2 ft[VP], fd[VP];
+              Vec<Tin>::pairs(ut[v], ft);
+              Vec<Tin>::pairs(ud[v], fd);
+#pragma unroll
+              for (int p = 0; p < VP; p += 2) {
+                ct0 = __fadd2_rn(ct0, ex2_pair(__ffma2_rn(ft[p], L2E, nmt)));
+                cd0 = __fadd2_rn(cd0, ex2_pair(__ffma2_rn(fd[p], L2E, nmd)));
+                ct1 = __fadd2_rn(ct1, ex2_pair(__ffma2_rn(ft[p + 1], L2E, nmt)));
+                cd1 = __fadd2_rn(cd1, ex2_pair(__ffma2_rn(fd[p + 1], L2E, nmd)));
+              }
+            }
+          }
+          const float st = (ct0.x + ct0.y) + (ct1.x + ct1.y);
+          const float sd = (cd0.x + cd0.y) + (cd1.x + cd1.y);
+          if (st <= 0x1p64f && sd <= 0x1p64f) {
+            at0 = __fadd2_rn(at0, ct0);
+            at1 = __fadd2_rn(at1, ct1);
+            ad0 = __fadd2_rn(ad0, cd0);
+            ad1 = __fadd2_rn(ad1, cd1);
+          } else {
+            exact = true;
+          }
+        }
+        if (exact) {
+#pragma unroll
+          for (int v = 0; v < kVPT; ++v) {
+            if (in[v]) {
+              raise(Vec<Tin>::vmax(ut[v]) * kLog2e, mt, at0, at1);
+              raise(Vec<Tin>::vmax(ud[v]) * kLog2e, md, ad0, ad1);
+              float2 ft[VP], fd[VP];
+              Vec<Tin>::pairs(ut[v], ft);
+              Vec<Tin>::pairs(ud[v], fd);
+              const float2 nmt = make_float2(-mt, -mt), nmd = make_float2(-md, -md);
+#pragma unroll
+              for (int p = 0; p < VP; p += 2) {
+                at0 = __fadd2_rn(at0, ex2_pair(__ffma2_rn(ft[p], L2E, nmt)));
+                ad0 = __fadd2_rn(ad0, ex2_pair(__ffma2_rn(fd[p], L2E, nmd)));
+                at1 = __fadd2_rn(at1, ex2_pair(__ffma2_rn(ft[p + 1], L2E, nmt)));
+                ad1 = __fadd2_rn(ad1, ex2_pair(__ffma2_rn(fd[p + 1], L2E, nmd)));
+              }
             }
           }
         }
