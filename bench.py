@@ -343,14 +343,53 @@ TV_SOURCES = (
 )
 
 
-def tv_source_sha256():
-    """Hash of the E2E-TV kernel sources (the counters below belong to it)."""
+def strip_c_comments(src):
+    """C/C++ source without its comments, whitespace runs collapsed to one
+    space (string and character literals kept as they are)."""
+    out, i, n, quote = [], 0, len(src), None
+    while i < n:
+        c = src[i]
+        if quote is None:
+            if src.startswith("//", i):
+                j = src.find("\n", i)
+                i = n if j < 0 else j
+                continue
+            if src.startswith("/*", i):
+                j = src.find("*/", i + 2)
+                i = n if j < 0 else j + 2
+                out.append(" ")
+                continue
+            if c in "\"'":
+                quote = c
+        elif c == "\\" and i + 1 < n:
+            out.append(src[i:i + 2])
+            i += 2
+            continue
+        elif c == quote:
+            quote = None
+        out.append(c)
+        i += 1
+    return " ".join("".join(out).split())
+
+
+def source_digest(texts):
+    """SHA-256 over sources with comments and layout removed: what the
+    compiler sees of them, so an edit of a comment keeps the digest."""
     import hashlib
     h = hashlib.sha256()
-    for rel in TV_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+    for t in texts:
+        h.update(strip_c_comments(t).encode())
+        h.update(b"\0")
     return h.hexdigest()
+
+
+def tv_source_sha256():
+    """Digest of the E2E-TV kernel sources (the counters below belong to it)."""
+    texts = []
+    for rel in TV_SOURCES:
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            texts.append(f.read())
+    return source_digest(texts)
 
 
 def _ncu_traffic():

@@ -94,3 +94,18 @@ def test_reference_arm_other_ranks_print_nothing():
                      env={"RANK": "1", "WORLD_SIZE": "2"})
     assert out.returncode == 0, out.stderr[-2000:]
     assert not [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_source_digest_ignores_comments_only():
+    src = ('// header\n#include "x.h"\nint f(int a) {  /* sum */\n'
+           '  const char* s = "a // b /* c */";\n  return a + \'/\';  // tail\n}\n')
+    d = bench.source_digest([src])
+    # comments and layout edited: same digest
+    moved = ('#include "x.h"\n/* new block\n comment */ int f(int a)\n{\n'
+             '  const char* s = "a // b /* c */"; return a + \'/\';\n}\n')
+    assert bench.source_digest([moved]) == d
+    # code edited (also inside a string literal): another digest
+    assert bench.source_digest([src.replace("a + ", "a - ")]) != d
+    assert bench.source_digest([src.replace("/* c */\";", "/* C */\";")]) != d
+    # file boundaries count
+    assert bench.source_digest([src, ""]) != d

@@ -16,10 +16,11 @@
 // The passes of consecutive tasks are pipelined: phase k interleaves pass A
 // of task k with pass C of task k - 1 chunk by chunk (A leads by kLag
 // chunks), then runs pass B of task k.  So each phase reads new rows from
-// DRAM while it writes the previous gradient row, the L2 holds about one
-// task's rows per CTA (pass C frees task k - 1's chunks as pass A brings in
-// task k's), and the branch handshake of task k - 1 has pass B of that task
-// and the first chunks of pass A of task k to complete in.
+// DRAM while it writes the previous gradient row, and the branch handshake
+// of task k - 1 has pass B of that task and the first chunks of pass A of
+// task k to complete in.  The price is L2 reuse distance: between pass A
+// of a task and its pass B the L2 also serves pass C of the previous task,
+// so part of pass B's and pass C's re-reads come from DRAM.
 //
 // Roles: one producer warp issues the 1-D bulk copies (TMA) of every chunk
 // ahead of the consumers (pass A at normal L2 priority, pass B evict-last,
