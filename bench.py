@@ -288,6 +288,9 @@ def run_gpu(args):
         attn_tflops = pb.flops / (attn_ms / 1e3) / 1e12
         clocks = _clock_summary(clk_path, local)
         traffic = _ncu_traffic() if wl == WORKLOAD else None  # counters of the 8B launch
+        # DRAM bytes actually moved per launch (ncu) over the live launch time:
+        # re-reads that miss L2 count here and not in `achieved`
+        dram_gbs = traffic / (tv_ms / 1e3) / 1e9 if traffic else None
         line = {
             "metric": METRIC,
             "value": value,
@@ -311,6 +314,8 @@ def run_gpu(args):
             "roofline": {"bound": "hbm", "kernel": "e2e_tv", "achieved": tv_gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": tv_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                         "dram_gbs": dram_gbs,
+                         "dram_frac": dram_gbs / peaks["hbm_gbs"] if dram_gbs else None,
                          "algorithmic_bytes_per_launch": pb.tv_bytes, "launch_ms": tv_ms,
                          "peak_src": peaks["src"]},
             "attention_roofline": {"bound": "tensor" if pb.acfg.dtype == "bf16" else "fp32 SIMT",
