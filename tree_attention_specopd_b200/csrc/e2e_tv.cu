@@ -16,9 +16,18 @@
 //   dz_d[n,u] = g_n q_u ([q_u < p_u] - s_n)
 // (d a / d z_u = sum_v [q_v<p_v] q_v (delta_vu - q_u) = q_u ([q_u<p_u] - s).)
 //
-// B200 design.  The kernel is HBM-bound: its algorithmic traffic is one
-// read of both logit rows and one write of the gradient, and it moves
-// exactly that.
+// B200 design.  The work is HBM-bound: its algorithmic traffic is one read
+// of both logit rows and one write of the gradient.  Two schedules, picked
+// by the host code at the end of this file:
+//  - whole-row (e2e_tv_row.cuh, the default for 16-byte aligned rows and W
+//    up to the SM count): one position per task, its rows streamed through
+//    a shared-memory ring three times with the passes of consecutive tasks
+//    pipelined;
+//  - slice (this file's kernel, the fallback): a position's rows cut into
+//    slices that stay in shared memory for all three passes, so it moves
+//    exactly the algorithmic bytes, at the price of a cross-CTA handshake
+//    per position and per branch.
+// The slice schedule:
 //  * Task = (position n, vocabulary slice c), NS slices per row.  A CTA
 //    (128 threads) holds one task: both rows' slice arrive by 1-D bulk copy
 //    (TMA) into its shared memory and stay there for all three passes.  Four
