@@ -18,6 +18,26 @@ def rel_err(x, ref):
     return float(np.max(np.abs(x - ref))) / den
 
 
+def assert_close_elementwise(x, ref, rtol, atol, what=""):
+    """Every element within |x - ref| <= rtol * |ref| + atol.
+
+    This is the per-element form of a relative tolerance: a small element is
+    held to its own magnitude, not to the largest element of the tensor
+    (atol only covers reference values at or near zero)."""
+    x = np.asarray(x, dtype=np.float64).ravel()
+    ref = np.asarray(ref, dtype=np.float64).ravel()
+    assert x.shape == ref.shape, (what, x.shape, ref.shape)
+    if ref.size == 0:
+        return
+    assert np.all(np.isfinite(x) == np.isfinite(ref)), f"{what}: non-finite pattern differs"
+    fin = np.isfinite(ref)
+    excess = np.abs(x[fin] - ref[fin]) - (rtol * np.abs(ref[fin]) + atol)
+    k = int(np.argmax(excess))
+    assert excess[k] <= 0, (f"{what}: element {np.flatnonzero(fin)[k]} = {x[fin][k]!r} vs "
+                            f"{ref[fin][k]!r} (|err| {abs(x[fin][k] - ref[fin][k]):.3e} > "
+                            f"{rtol:g}*|ref| + {atol:g})")
+
+
 def dev_tensor(x, dtype, device="cuda"):
     """Host float array -> CUDA tensor of `dtype` ("f32" or "bf16").  bf16
     values must already be bf16-exact (synth rounds them)."""

@@ -153,7 +153,7 @@ def test_anchor_out_of_range_bf16(lib):
     assert lib.specopd_get_device_status() & lib.DEV_ANCHOR_RANGE
 
 
-@pytest.mark.parametrize("name,nsample", [("8b", None), ("long", 6), ("packed", 6)])
+@pytest.mark.parametrize("name,nsample", [("8b", None), ("long", 64), ("packed", 64)])
 def test_full_size_workloads(lib, name, nsample):
     # The full workloads, in the launch configuration the benchmark times;
     # the oracle checks every branch of the 8B shape and a seeded sample of

@@ -15,7 +15,7 @@ import synth
 from oracle import attention as oatt
 from oracle import tree as otree
 from oracle import tv as otv
-from tests._util import dev_tensor, rel_err, to_np
+from tests._util import assert_close_elementwise, dev_tensor, rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -105,6 +105,14 @@ def _attn_run(lib, inp, rope_base=10000.0):
     return to_np(out), to_np(lse)
 
 
+# fp32 attention outputs: 1e-5 relative per element, plus an absolute floor
+# for outputs near zero.  An output is a softmax-weighted mean of unit-scale
+# values; the RoPE angles are evaluated in fp32 on the GPU (about 1e-7
+# relative on the rotated q/k), so scores, and hence every output, carry an
+# absolute error of order 1e-7 whatever the output's own size.
+ATT32_RTOL, ATT32_ATOL = 1e-5, 1e-6
+
+
 def _attn_ref(inp):
     cfg = inp.cfg
     return oatt.branch_attention_unrolled_dense(inp.q_br, inp.k_br, inp.v_br, inp.k_tr, inp.v_tr,
@@ -118,6 +126,7 @@ def test_attention_tiny_fp32(lib):
     ref = _attn_ref(inp)
     assert out.shape == ref.shape == (12, 4, 64)
     assert rel_err(out, ref) < 1e-5
+    assert_close_elementwise(out, ref, ATT32_RTOL, ATT32_ATOL, "out")
     assert _status(lib) == 0
 
 
@@ -134,7 +143,9 @@ def test_attention_fp32_edges(lib, S, T, B, W, Hq, Hkv, D, anchors):
         assert out.shape[0] == 0
         return
     out, _ = _attn_run(lib, inp)
-    assert rel_err(out, _attn_ref(inp)) < 1e-5
+    ref = _attn_ref(inp)
+    assert rel_err(out, ref) < 1e-5
+    assert_close_elementwise(out, ref, ATT32_RTOL, ATT32_ATOL, "out")
     assert _status(lib) == 0
 
 
@@ -178,9 +189,17 @@ def _tv_run(lib, zt, zd, nb, W, dtype, grad_dtype="f32", target_row=None, zt_row
     return res
 
 
+# fp32 outputs: 1e-5 relative per element, with a 1e-7 floor for reference
+# values at or near zero (disjoint supports, late prefix products of
+# low-overlap branches).  Gradient rows are compared normwise per row: near a
+# tie q_v = p_v the fp32 kernel and the fp64 oracle may take different sides
+# of the subgradient of min, which moves single elements of a row.
+TV_RTOL, TV_ATOL = 1e-5, 1e-7
+
+
 def _check_tv(res, ref, rows=None, grad=True):
-    assert rel_err(to_np(res["a"]), ref["a"]) < 1e-5
-    assert rel_err(to_np(res["prefix"]), ref["prefix"]) < 1e-5
+    assert_close_elementwise(to_np(res["a"]), ref["a"], TV_RTOL, TV_ATOL, "a")
+    assert_close_elementwise(to_np(res["prefix"]), ref["prefix"], TV_RTOL, TV_ATOL, "prefix")
     assert abs(res["loss"].item() - ref["loss"]) <= 1e-4 * abs(ref["loss"]) + 1e-7
     assert abs(res["numer"].item() - ref["numer"]) <= 1e-5 * abs(ref["numer"]) + 1e-7
     if grad:
@@ -347,7 +366,7 @@ def test_tv_no_grad_many_tasks(lib):
     assert rn["grad"] is None
     for k in ("a", "prefix", "loss", "numer"):
         assert torch.equal(rg[k], rn[k]), k
-    assert rel_err(to_np(rn["a"]), ref["a"]) < 1e-5
+    assert_close_elementwise(to_np(rn["a"]), ref["a"], TV_RTOL, TV_ATOL, "a")
     assert abs(rn["loss"].item() - ref["loss"]) <= 1e-4 * abs(ref["loss"]) + 1e-7
 
 

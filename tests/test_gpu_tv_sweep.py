@@ -10,7 +10,9 @@ branches (a branch's gradient needs only its own W overlaps and the global
 position count).
 
 Tolerances (fp32 accumulation against fp64): overlaps and prefix products
-1e-5 relative, loss 1e-4 relative, gradient rows 1e-3 relative.
+1e-5 relative per element (1e-7 floor for values at or near zero), loss
+1e-4 relative, gradient rows 1e-3 relative (normwise per row: near-ties of
+q and p may take the other side of the subgradient of min).
 """
 
 import numpy as np
@@ -19,7 +21,7 @@ import torch
 
 import synth
 from oracle import tv as otv
-from tests._util import rel_err, to_np
+from tests._util import assert_close_elementwise, rel_err, to_np
 
 CHUNK = 256  # positions per host-side chunk
 
@@ -53,9 +55,10 @@ def test_tv_overlap_sweep_full_size(lib, sigma_index):
     assert lib.specopd_get_device_status() == 0
 
     a = to_np(res["a"]).astype(np.float64)
-    assert rel_err(a, a_ref) < 1e-5
+    assert_close_elementwise(a, a_ref, 1e-5, 1e-7, "a")
     P_ref = otv.prefix_products(a_ref.reshape(cfg.nbranch, W))
-    assert rel_err(to_np(res["prefix"]).reshape(cfg.nbranch, W), P_ref) < 1e-5
+    assert_close_elementwise(to_np(res["prefix"]).reshape(cfg.nbranch, W), P_ref, 1e-5, 1e-7,
+                             "prefix")
     loss_ref = otv.loss_from_overlaps(a_ref.reshape(cfg.nbranch, W), N)
     assert abs(res["loss"].item() - loss_ref) <= 1e-4 * abs(loss_ref) + 1e-7
 
@@ -66,6 +69,8 @@ def test_tv_overlap_sweep_full_size(lib, sigma_index):
     assert ident and disj
     assert np.all(np.abs(a[ident] - 1.0) < 1e-5)
     assert np.all(a_ref[disj] < 1e-3) and np.all(a[disj] < 1e-3)
+    assert_close_elementwise(a[disj], a_ref[disj], 1e-5, 1e-7, "a (disjoint rows)")
+    assert_close_elementwise(a[ident], a_ref[ident], 1e-5, 1e-7, "a (identical rows)")
 
     # gradient rows of sampled whole branches, one of them holding an
     # identical row and one a disjoint row
