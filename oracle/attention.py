@@ -23,6 +23,13 @@ the branch tokens, with textbook causal attention; no tiling, packing or
 online softmax.  ``packed_tree_attention`` is a second formulation (one
 packed sequence with an explicit dense tree mask) used only to pin
 packed == unrolled.
+
+``trunk_prefill`` is the step before the branch pass: the shared prefix
+computed once (review §3.2(a): the trunk K/V is computed once and cached;
+the aimodeling.com page: the trunk is prefilled once and its branches reuse
+it).  Every trunk position of every sequence is a query of plain causal
+attention over its own sequence, with RoPE at the trunk position, and the
+rotated trunk keys are the K cache the branch pass reads.
 """
 
 from __future__ import annotations
@@ -158,3 +165,37 @@ def packed_tree_attention(q_br, k_br, v_br, k_tr_raw, v_tr, parent, sem_pos,
         s = np.where(mask, s, -np.inf)
         out[:, h, :] = softmax_rows(s) @ v_all[:, g]
     return out
+
+
+def trunk_prefill(q_tr, k_tr_raw, v_tr, cu_trunk, base, scale=None):
+    """Causal self-attention over each trunk sequence, with RoPE.
+
+    q_tr [T_tot, Hq, D], k_tr_raw / v_tr [T_tot, Hkv, D] (any float dtype,
+    computed in fp64; K not rotated).  Sequence s owns rows
+    cu_trunk[s] .. cu_trunk[s+1]-1 at positions 0 .. T_s-1; a query at
+    position t sees the keys of its own sequence at positions <= t.
+    Returns (out [T_tot, Hq, D], k_cache [T_tot, Hkv, D]), both fp64, where
+    k_cache is K rotated at the trunk positions.
+    """
+    q_tr = np.asarray(q_tr, dtype=np.float64)
+    k_tr_raw = np.asarray(k_tr_raw, dtype=np.float64)
+    v_tr = np.asarray(v_tr, dtype=np.float64)
+    cu = [int(c) for c in cu_trunk]
+    Hq, D = q_tr.shape[1], q_tr.shape[2]
+    Hkv = k_tr_raw.shape[1]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = np.empty_like(q_tr)
+    k_cache = np.empty_like(k_tr_raw)
+    for s in range(len(cu) - 1):
+        rows = slice(cu[s], cu[s + 1])
+        pos = np.arange(cu[s + 1] - cu[s], dtype=np.int64)
+        k_rot = rope(k_tr_raw[rows], pos, base)
+        q_rot = rope(q_tr[rows], pos, base)
+        k_cache[rows] = k_rot
+        for h in range(Hq):
+            g = h // G
+            out[rows, h, :] = causal_attention(q_rot[:, h], k_rot[:, g], v_tr[rows, g], pos, pos,
+                                               scale)
+    return out, k_cache

@@ -157,3 +157,76 @@ def test_rows_are_convex_combinations_of_visible_values():
     c["vt"][:] = 0.25
     c["vb"][:] = 0.25
     np.testing.assert_allclose(_unrolled(c), 0.25, rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- trunk prefill
+
+def _prefill_case(rng, T, Hq, Hkv, D):
+    cu = np.concatenate([[0], np.cumsum(T)]).astype(int)
+    n = int(cu[-1])
+    return cu, _rand(rng, n, Hq, D), _rand(rng, n, Hkv, D), _rand(rng, n, Hkv, D)
+
+
+def test_prefill_single_sequence_is_textbook_causal_attention():
+    # One sequence, Hq = Hkv = 1: torch SDPA with is_causal on the rotated
+    # inputs (a library routine, independent of the oracle's own softmax).
+    rng = np.random.default_rng(11)
+    cu, q, k, v = _prefill_case(rng, [37], 1, 1, 16)
+    out, kc = att.trunk_prefill(q, k, v, cu, 1e4)
+    pos = np.arange(37)
+    qr = att.rope(q, pos, 1e4)[:, 0]
+    kr = att.rope(k, pos, 1e4)[:, 0]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(qr)[None], torch.tensor(kr)[None], torch.tensor(v[:, 0])[None],
+        is_causal=True)[0].numpy()
+    np.testing.assert_allclose(out[:, 0], ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(kc[:, 0], kr)
+
+
+def test_prefill_first_row_is_its_own_value():
+    # Position 0 sees only itself: its output is v_0 for every head.
+    rng = np.random.default_rng(12)
+    cu, q, k, v = _prefill_case(rng, [5, 9, 1], 4, 2, 8)
+    out, _ = att.trunk_prefill(q, k, v, cu, 1e4)
+    for s in range(3):
+        r = cu[s]
+        np.testing.assert_allclose(out[r], np.repeat(v[r], 2, axis=0), rtol=0, atol=1e-15)
+
+
+def test_prefill_sequences_do_not_see_each_other():
+    # A packed batch gives each sequence exactly its own prefill, and keys
+    # after a row's position cannot move it.
+    rng = np.random.default_rng(13)
+    T = [6, 11, 4]
+    cu, q, k, v = _prefill_case(rng, T, 2, 1, 8)
+    out, kc = att.trunk_prefill(q, k, v, cu, 1e4)
+    for s in range(3):
+        rows = slice(cu[s], cu[s + 1])
+        o1, k1 = att.trunk_prefill(q[rows], k[rows], v[rows], [0, T[s]], 1e4)
+        np.testing.assert_array_equal(out[rows], o1)
+        np.testing.assert_array_equal(kc[rows], k1)
+    k2, v2 = k.copy(), v.copy()
+    k2[cu[1] + 5:] += 50.0   # sequence 1 from position 5 on, and everything after it
+    v2[cu[1] + 5:] -= 9.0
+    out2, _ = att.trunk_prefill(q, k2, v2, cu, 1e4)
+    np.testing.assert_array_equal(out2[: cu[1] + 5], out[: cu[1] + 5])
+    assert not np.array_equal(out2[cu[1] + 5], out[cu[1] + 5])
+
+
+def test_prefill_then_branch_equals_one_longer_prefill():
+    # Review §3.2(a): the branch pass reuses the cached trunk.  A branch
+    # scored over the prefilled cache gives the same rows as prefilling the
+    # linear sequence trunk[0..a] followed by the branch tokens: its last W-1
+    # rows.  The two sides use different formulations (packed tree mask
+    # against per-sequence causal attention).
+    rng = np.random.default_rng(14)
+    T, a, W, Hq, Hkv, D = 20, 12, 4, 2, 1, 8
+    c = _case(rng, 1, [T], 1, W, Hq, Hkv, D, anchors=[a])
+    parent, sem_pos, _ = tree.tree_build(c["cu"], c["anchors"], 1, W)
+    branch = att.packed_tree_attention(c["q"], c["kb"], c["vb"], c["kt"], c["vt"], parent,
+                                       sem_pos, T, 1e4)
+    q_seq = np.concatenate([_rand(rng, a + 1, Hq, D), c["q"]])
+    k_seq = np.concatenate([c["kt"][: a + 1], c["kb"]])
+    v_seq = np.concatenate([c["vt"][: a + 1], c["vb"]])
+    out, _ = att.trunk_prefill(q_seq, k_seq, v_seq, [0, a + W], 1e4)
+    np.testing.assert_allclose(out[a + 1:], branch, rtol=1e-12, atol=1e-12)
