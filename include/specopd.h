@@ -199,6 +199,42 @@ specopd_status specopd_tree_attn(const specopd_attn_desc* desc,
                                  size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Trunk prefill: [review §3.2(a)] (the trunk -- prompt plus reference
+ * response -- is computed once and its K/V cached; every branch then reads
+ * that cache) and the aimodeling.com news page (the trunk is prefilled once
+ * and shared by all of its branches).  The step before specopd_tree_attn:
+ * plain causal self-attention of every trunk token over its own sequence.
+ *
+ * For trunk row t of sequence s (position p = t - cu_trunk[s]) and query
+ * head h (kv head h / (Hq/Hkv)):
+ *   keys      = trunk rows cu_trunk[s] .. t            (p + 1 keys)
+ *   out[t,h,:] = softmax(scale * q' . k'^T) v,   scale = 1/sqrt(D) unless set
+ * with q' and k' rotated at their positions within their sequence (the RoPE
+ * convention of specopd_rope_apply).  Sequences never see each other.
+ *
+ * desc       the same descriptor as specopd_tree_attn (B and W are not used)
+ * q_tr       [T_tot, Hq, D] trunk queries, NOT rotated
+ * k_tr       [T_tot, Hkv, D] IN: trunk keys, not rotated.  OUT: the K cache,
+ *            rotated in place -- the k_tr argument of specopd_tree_attn.
+ * v_tr       [T_tot, Hkv, D] trunk values (the V cache as it is)
+ * cu_trunk / cu_trunk_host  device / host int32[S+1]
+ * out        [T_tot, Hq, D] (dtype); row cu_trunk[s] + a is the anchor row
+ *            whose target output scores the first token of a branch at a
+ * lse        optional fp32 [T_tot, Hq] natural-log sum-exp, or NULL
+ * The bf16 path runs on the tensor cores (the kernel of specopd_tree_attn
+ * with the trunk rows as queries); fp32 uses the SIMT kernel.
+ */
+size_t specopd_trunk_prefill_workspace_size(const specopd_attn_desc* desc,
+                                            const int32_t* cu_trunk_host);
+
+specopd_status specopd_trunk_prefill(const specopd_attn_desc* desc,
+                                     const void* q_tr, void* k_tr,
+                                     const void* v_tr, const int32_t* cu_trunk,
+                                     const int32_t* cu_trunk_host, void* out,
+                                     float* lse, void* workspace, size_t ws_bytes,
+                                     void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* E2E-TV loss: [review §1.1] and [review §3.3] (single-draft acceptance
  * probability = overlap of the two distributions = 1 - TV(p, q); the loss is
  * built from prefix products of the overlaps within each branch; target mass
@@ -255,6 +291,26 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* desc,
                               void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Distributed normalisation of the E2E-TV loss: [review §3.2], its paragraph
+ * on numerical consistency (numerators and counts are gathered separately
+ * over the ranks and the loss normalised once, so the weight of a position
+ * does not depend on how many positions its rank scored).
+ *
+ * When the branches of a batch are sharded over ranks, every rank calls
+ * specopd_e2e_tv on its own branches with norm_count = the GLOBAL position
+ * count (its gradient then already carries the global 1/N), the ranks sum
+ * their `numer` outputs (one all-reduce of one double), and this call
+ * finishes the loss on the device:
+ *   loss = 1 - numer_sum / norm_count
+ * numer_sum   device fp64[1]: the sum over ranks of specopd_e2e_tv's numer
+ * norm_count  the global position count, > 0 (the one every rank passed)
+ * loss        device fp32[1] (out)
+ * loss64      device fp64[1] (out), or NULL
+ */
+specopd_status specopd_e2e_tv_finalize(const double* numer_sum, int64_t norm_count,
+                                       float* loss, double* loss64, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* E2E-TV for callers that cannot allocate device memory.  The paper has no
  * counterpart: this is an interface addition of this library.
  *
@@ -266,11 +322,18 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* desc,
  * workspace) and allocates nothing: its scratch is a fixed array of
  * SPECOPD_E2E_TV_STATIC_SCRATCH_BYTES in the library's device image, held by
  * every GPU that loads the library until the process exits.
- *   - Size limit: returns SPECOPD_ERR_WORKSPACE, launching nothing, when
- *     specopd_e2e_tv_workspace_size(desc) exceeds the array (8 MiB: about
- *     28,000 positions at a 151,936-token bf16 vocabulary and W = 8).
+ *   - Size limit: returns SPECOPD_ERR_WORKSPACE, launching nothing, when the
+ *     scratch of the schedule this call runs exceeds the array (8 MiB).  With
+ *     16-byte aligned rows and W up to the SM count (the whole-row schedule)
+ *     that is about 10 bytes per position plus a few per branch: any problem
+ *     up to about 800,000 positions fits.  The slice fallback (unaligned rows) needs about
+ *     24 bytes per position and vocabulary slice: about 29,000 positions at a
+ *     151,936-token bf16 vocabulary.
  *   - The first call on each device resolves the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     (cudaGetSymbolAddress) and keeps it for the life of the process; make
+ *     that first call before any stream capture, and do not use this entry
+ *     point across a reset of the device (cudaDeviceReset), which can move
+ *     the array.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents (each call clears what must start at zero).  Calls that
  *     overlap on the GPU -- other streams, other host threads -- race on it:
@@ -284,6 +347,28 @@ specopd_status specopd_e2e_tv_noalloc(const specopd_tv_desc* desc,
                                       const void* z_draft, float* a, float* prefix,
                                       float* loss, double* numer, void* grad_draft,
                                       void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Testing hook: host-driven fault injection.  The paper has no counterpart.
+ *
+ * Lets a test make a bounded device-side wait run out on purpose, without
+ * faulting, trapping or hanging the GPU, to check the library's wind-down:
+ *   withhold_position  >= 0: in E2E-TV calls that use the whole-row schedule
+ *                      (the default for 16-byte aligned rows and W up to the
+ *                      SM count), the scorer of that supervised position never
+ *                      publishes its overlap, so every position of its branch
+ *                      waits for it in vain; -1 (the default) turns this off.
+ *   branch_wait_limit_ns  limit of those branch waits; 0 (the default) keeps
+ *                      the normal limit of 2 s.
+ * When such a wait runs out the kernel sets SPECOPD_DEV_TIMEOUT, writes NaN
+ * to the outputs of the affected branch (and the loss), finishes every other
+ * branch normally and returns.  The setting is per device (the current one),
+ * applies to calls launched after it, and stays until changed: reset it with
+ * (-1, 0).  Call it only while no E2E-TV call is running on the device.
+ * Returns SPECOPD_ERR_CUDA if the setting could not be written.
+ */
+specopd_status specopd_debug_fault_injection(int64_t withhold_position,
+                                             uint64_t branch_wait_limit_ns);
 
 #ifdef __cplusplus
 }

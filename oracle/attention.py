@@ -167,7 +167,7 @@ def packed_tree_attention(q_br, k_br, v_br, k_tr_raw, v_tr, parent, sem_pos,
     return out
 
 
-def trunk_prefill(q_tr, k_tr_raw, v_tr, cu_trunk, base, scale=None):
+def trunk_prefill(q_tr, k_tr_raw, v_tr, cu_trunk, base, scale=None, rows=None):
     """Causal self-attention over each trunk sequence, with RoPE.
 
     q_tr [T_tot, Hq, D], k_tr_raw / v_tr [T_tot, Hkv, D] (any float dtype,
@@ -175,7 +175,9 @@ def trunk_prefill(q_tr, k_tr_raw, v_tr, cu_trunk, base, scale=None):
     cu_trunk[s] .. cu_trunk[s+1]-1 at positions 0 .. T_s-1; a query at
     position t sees the keys of its own sequence at positions <= t.
     Returns (out [T_tot, Hq, D], k_cache [T_tot, Hkv, D]), both fp64, where
-    k_cache is K rotated at the trunk positions.
+    k_cache is K rotated at the trunk positions.  With ``rows`` (packed row
+    indices), only those rows of ``out`` are computed (the others are NaN),
+    each with the same formula over its own visible keys.
     """
     q_tr = np.asarray(q_tr, dtype=np.float64)
     k_tr_raw = np.asarray(k_tr_raw, dtype=np.float64)
@@ -186,16 +188,23 @@ def trunk_prefill(q_tr, k_tr_raw, v_tr, cu_trunk, base, scale=None):
     G = Hq // Hkv
     if scale is None:
         scale = 1.0 / np.sqrt(D)
-    out = np.empty_like(q_tr)
+    out = np.full_like(q_tr, np.nan)
     k_cache = np.empty_like(k_tr_raw)
+    want = None if rows is None else np.asarray(sorted(set(int(r) for r in rows)), dtype=np.int64)
     for s in range(len(cu) - 1):
-        rows = slice(cu[s], cu[s + 1])
+        seq = slice(cu[s], cu[s + 1])
         pos = np.arange(cu[s + 1] - cu[s], dtype=np.int64)
-        k_rot = rope(k_tr_raw[rows], pos, base)
-        q_rot = rope(q_tr[rows], pos, base)
-        k_cache[rows] = k_rot
+        k_rot = rope(k_tr_raw[seq], pos, base)
+        k_cache[seq] = k_rot
+        if want is None:
+            sel = pos
+        else:
+            sel = want[(want >= cu[s]) & (want < cu[s + 1])] - cu[s]
+            if sel.size == 0:
+                continue
+        q_rot = rope(q_tr[seq][sel], sel, base)
         for h in range(Hq):
             g = h // G
-            out[rows, h, :] = causal_attention(q_rot[:, h], k_rot[:, g], v_tr[rows, g], pos, pos,
-                                               scale)
+            out[cu[s] + sel, h, :] = causal_attention(q_rot[:, h], k_rot[:, g], v_tr[seq, g], sel,
+                                                      pos, scale)
     return out, k_cache

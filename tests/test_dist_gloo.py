@@ -3,9 +3,9 @@ distributed normalisation of the loss (SpecOPD review §3.2: numerators and
 counts gathered separately) reproduce the single-process oracle exactly,
 including when the ranks hold different numbers of branches.
 
-The per-rank compute here is the oracle (CPU); on GPUs the same host code
-wraps specopd_e2e_tv (bench.py), whose numer/norm_count arguments are the
-quantities exchanged below.
+The per-rank compute here is the oracle (CPU), and the loss is finished on
+the host; tests/test_gpu_dist.py runs the same exchange around the library
+(specopd_e2e_tv per shard, specopd_e2e_tv_finalize after the sum).
 """
 
 import os
@@ -47,8 +47,8 @@ def _worker(rank, world, port, nb, W, V, out_q):
         n_global = sdist.global_count(cnt * W)
         res = otv.e2e_tv(zt[rows], None, zd[rows], cnt, W, norm_count=n_global)
         numer = torch.tensor([res["numer"]], dtype=torch.float64)
-        loss = sdist.global_loss(numer, n_global)
-        out_q.put((rank, start, cnt, float(loss.item()), res["g"].tolist(), n_global))
+        loss = 1.0 - sdist.global_numer(numer).item() / n_global
+        out_q.put((rank, start, cnt, float(loss), res["g"].tolist(), n_global))
     finally:
         dist.destroy_process_group()
 

@@ -230,3 +230,15 @@ def test_prefill_then_branch_equals_one_longer_prefill():
     v_seq = np.concatenate([c["vt"][: a + 1], c["vb"]])
     out, _ = att.trunk_prefill(q_seq, k_seq, v_seq, [0, a + W], 1e4)
     np.testing.assert_allclose(out[a + 1:], branch, rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_sampled_rows_equal_full_rows():
+    rng = np.random.default_rng(15)
+    cu, q, k, v = _prefill_case(rng, [9, 30, 4], 4, 2, 8)
+    full, kc = att.trunk_prefill(q, k, v, cu, 1e4)
+    rows = [0, 8, 9, 25, 38, 42]
+    part, kc2 = att.trunk_prefill(q, k, v, cu, 1e4, rows=rows)
+    np.testing.assert_allclose(part[rows], full[rows], rtol=1e-12, atol=1e-13)  # BLAS blocking
+    np.testing.assert_array_equal(kc2, kc)
+    others = np.setdiff1d(np.arange(cu[-1]), rows)
+    assert np.all(np.isnan(part[others]))

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import synth
-from tests._util import dev_tensor, rel_err, to_np
+from tests._util import assert_close_elementwise, dev_tensor, rel_err, to_np
 from tree_attention_specopd_b200 import api
 
 pytestmark = pytest.mark.gpu
@@ -27,8 +27,8 @@ def _outputs(N, V, grad_dtype=torch.float32):
 
 
 def _compare(got, ref):
-    assert rel_err(to_np(got["a"]), to_np(ref["a"])) < 1e-5
-    assert rel_err(to_np(got["prefix"]), to_np(ref["prefix"])) < 1e-5
+    assert_close_elementwise(to_np(got["a"]), to_np(ref["a"]), 1e-5, 1e-7, "a")
+    assert_close_elementwise(to_np(got["prefix"]), to_np(ref["prefix"]), 1e-5, 1e-7, "prefix")
     assert abs(got["loss"].item() - ref["loss"].item()) <= 1e-4 * abs(ref["loss"].item())
     assert abs(got["numer"].item() - ref["numer"].item()) <= 1e-5 * abs(ref["numer"].item())
     g, gr = to_np(got["grad"]), to_np(ref["grad"])
@@ -72,8 +72,9 @@ def test_noalloc_matches_workspace_entry_point(nb, W, V, dtype, gather):
 
 
 def test_noalloc_rejects_sizes_beyond_the_array():
-    # 800,000 positions need more scratch than the fixed array holds.
-    desc = api.tv_desc(200_000, 4, 16, 800_000, "f32", "f32", True)
+    # A million positions need more scratch than the fixed array holds, even
+    # on the schedules that need the least (about 10 bytes per position).
+    desc = api.tv_desc(250_000, 4, 16, 1_000_000, "f32", "f32", True)
     assert api.specopd_e2e_tv_workspace_size(desc) > api.E2E_TV_STATIC_SCRATCH_BYTES
     dummy = torch.empty(1, device="cuda")
     with pytest.raises(api.SpecopdError) as ei:

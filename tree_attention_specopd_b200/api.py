@@ -83,6 +83,12 @@ def load(path: str = LIB_PATH):
     lib.specopd_tree_attn.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, i32p,
                                       ctypes.POINTER(ctypes.c_int32), i32p, i32p, vp, f32p,
                                       vp, csize, vp]
+    lib.specopd_trunk_prefill_workspace_size.restype = csize
+    lib.specopd_trunk_prefill_workspace_size.argtypes = [ctypes.POINTER(AttnDesc),
+                                                         ctypes.POINTER(ctypes.c_int32)]
+    lib.specopd_trunk_prefill.restype = cint
+    lib.specopd_trunk_prefill.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, i32p,
+                                          ctypes.POINTER(ctypes.c_int32), vp, f32p, vp, csize, vp]
     lib.specopd_e2e_tv_workspace_size.restype = csize
     lib.specopd_e2e_tv_workspace_size.argtypes = [ctypes.POINTER(TVDesc)]
     lib.specopd_e2e_tv.restype = cint
@@ -91,6 +97,10 @@ def load(path: str = LIB_PATH):
     lib.specopd_e2e_tv_noalloc.restype = cint
     lib.specopd_e2e_tv_noalloc.argtypes = [ctypes.POINTER(TVDesc), vp, i32p, vp, f32p, f32p,
                                            f32p, f64p, vp, vp]
+    lib.specopd_e2e_tv_finalize.restype = cint
+    lib.specopd_e2e_tv_finalize.argtypes = [f64p, ctypes.c_int64, f32p, f64p, vp]
+    lib.specopd_debug_fault_injection.restype = cint
+    lib.specopd_debug_fault_injection.argtypes = [ctypes.c_int64, ctypes.c_uint64]
     _lib = lib
     return lib
 
@@ -188,6 +198,28 @@ def specopd_tree_attn(desc, q_br, k_br, v_br, k_tr, v_tr, cu_trunk_dev, cu_trunk
     return out
 
 
+def specopd_trunk_prefill_workspace_size(desc, cu_trunk) -> int:
+    cu_arr, _ = _cu_host(cu_trunk)
+    return int(load().specopd_trunk_prefill_workspace_size(ctypes.byref(desc), cu_arr))
+
+
+def specopd_trunk_prefill(desc, q_tr, k_tr, v_tr, cu_trunk_dev, cu_trunk_host, out=None, lse=None,
+                          workspace=None, stream=None):
+    """Causal attention of every trunk row over its own sequence; k_tr is
+    rotated in place (it becomes the K cache).  Returns out [T_tot, Hq, D]."""
+    cu_arr, _ = _cu_host(cu_trunk_host)
+    if out is None:
+        out = torch.empty_like(q_tr)
+    if workspace is None:
+        n = specopd_trunk_prefill_workspace_size(desc, cu_trunk_host)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q_tr.device)
+    _check(load().specopd_trunk_prefill(ctypes.byref(desc), _ptr(q_tr), _ptr(k_tr), _ptr(v_tr),
+                                        _ptr(cu_trunk_dev), cu_arr, _ptr(out), _ptr(lse),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+           "trunk_prefill")
+    return out
+
+
 def tv_desc(nbranch, W, V, rows_target, logit_dtype, grad_dtype="f32", compute_grad=True,
             norm_count=0):
     def code(d):
@@ -224,6 +256,24 @@ def specopd_e2e_tv(desc, z_target, target_row, z_draft, a=None, prefix=None, los
                                  _ptr(grad), _ptr(workspace), workspace.numel(), _stream(stream)),
            "e2e_tv")
     return {"a": a, "prefix": prefix, "loss": loss, "numer": numer, "grad": grad}
+
+
+def specopd_e2e_tv_finalize(numer_sum, norm_count, loss=None, loss64=None, stream=None):
+    """loss = 1 - numer_sum / norm_count on the device (numer_sum: the fp64
+    sum over ranks of specopd_e2e_tv's numer).  Returns the fp32 loss tensor."""
+    if loss is None:
+        loss = torch.empty(1, dtype=torch.float32, device=numer_sum.device)
+    _check(load().specopd_e2e_tv_finalize(_ptr(numer_sum), int(norm_count), _ptr(loss),
+                                          _ptr(loss64), _stream(stream)), "e2e_tv_finalize")
+    return loss
+
+
+def specopd_debug_fault_injection(withhold_position=-1, branch_wait_limit_ns=0):
+    """Testing hook: make the E2E-TV scorer of one supervised position skip
+    publishing its overlap, and shorten the branch waits that then run out
+    (see include/specopd.h).  (-1, 0) turns it off."""
+    _check(load().specopd_debug_fault_injection(int(withhold_position), int(branch_wait_limit_ns)),
+           "debug_fault_injection")
 
 
 E2E_TV_STATIC_SCRATCH_BYTES = 8 << 20

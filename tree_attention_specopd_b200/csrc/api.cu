@@ -68,15 +68,28 @@ struct AttnWs {
   size_t q_off, k_off, tail_off, total;
 };
 
-AttnWs attn_ws_layout(const AttnProblem& p) {
+// fp32 (SIMT kernel): rotated copies of the branch q and k, rotated once by
+// a RoPE launch.  bf16 (tensor-core kernel): the split-KV partials only (the
+// kernel rotates q and k in shared memory).
+// Trunk prefill: fp32 keeps the rotated trunk queries, bf16 the split-KV
+// partials.
+AttnWs attn_ws_layout(const AttnProblem& p, bool prefill = false) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   AttnWs w;
   w.q_off = 0;
-  w.k_off = up((size_t)p.R * p.Hq * p.D * elt(p.dtype));
-  w.tail_off = up(w.k_off + (size_t)p.R * p.Hkv * p.D * elt(p.dtype));
-  size_t tail = 0;
-  if (p.dtype == SPECOPD_BF16) tail = attn_sm100_workspace(p);
-  w.total = up(w.tail_off + tail);
+  if (p.dtype == SPECOPD_BF16) {
+    w.k_off = 0;
+    w.tail_off = 0;
+    w.total = up(attn_sm100_workspace(p, prefill));
+  } else if (prefill) {
+    w.k_off = 0;
+    w.tail_off = up((size_t)p.T_tot * p.Hq * p.D * elt(p.dtype));
+    w.total = w.tail_off;
+  } else {
+    w.k_off = up((size_t)p.R * p.Hq * p.D * elt(p.dtype));
+    w.tail_off = up(w.k_off + (size_t)p.R * p.Hkv * p.D * elt(p.dtype));
+    w.total = w.tail_off;
+  }
   if (w.total < 256) w.total = 256;
   return w;
 }
@@ -116,6 +129,33 @@ specopd_status tv_problem(const specopd_tv_desc* d, TVProblem& p) {
   // Slices per row (each CTA holds one slice of both rows in shared memory).
   if (tv_slice_count(p) > kTVMaxSlices || d->W > kTVMaxW) return SPECOPD_ERR_UNSUPPORTED;
   return SPECOPD_OK;
+}
+
+// E2E-TV after host validation.  The workspace must hold
+// specopd_e2e_tv_workspace_size bytes, or, with exact_need, what the schedule
+// picked for these pointers needs (the allocation-free entry point, whose
+// scratch is fixed).
+specopd_status e2e_tv_checked(const specopd_tv_desc* d, const void* z_target,
+                              const int32_t* target_row, const void* z_draft, float* a,
+                              float* prefix, float* loss, double* numer, void* grad_draft,
+                              void* workspace, size_t ws_bytes, void* stream, bool exact_need) {
+  TVProblem p;
+  specopd_status s = tv_problem(d, p);
+  if (s != SPECOPD_OK) return s;
+  if (!z_target || !z_draft || !a || !prefix || !loss) return SPECOPD_ERR_INVALID_ARG;
+  if (p.compute_grad && !grad_draft) return SPECOPD_ERR_INVALID_ARG;
+  if (!target_row && p.rows_target < p.N) return SPECOPD_ERR_INVALID_ARG;
+  if (!workspace) return SPECOPD_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SPECOPD_ERR_UNSUPPORTED;
+  s = check_device();
+  if (s != SPECOPD_OK) return s;
+  void* grad = p.compute_grad ? grad_draft : nullptr;
+  const size_t need = exact_need ? tv_workspace_for_call(p, z_target, z_draft, grad) : tv_workspace(p);
+  if (ws_bytes < need) return SPECOPD_ERR_WORKSPACE;
+  cudaError_t e = launch_e2e_tv(p, z_target, target_row, z_draft, a, prefix, loss, numer, grad,
+                                workspace, ws_bytes, as_stream(stream));
+  if (e == cudaErrorInvalidConfiguration) { cudaGetLastError(); return SPECOPD_ERR_UNSUPPORTED; }
+  return cuda_status(e);
 }
 
 }  // namespace
@@ -217,22 +257,75 @@ specopd_status specopd_tree_attn(const specopd_attn_desc* d, const void* q_br, c
   if (s != SPECOPD_OK) return s;
   cudaStream_t st = as_stream(stream);
   char* ws = reinterpret_cast<char*>(workspace);
-  void* q_rot = ws + L.q_off;
-  void* k_rot = ws + L.k_off;
   double theta[128];
   rope_theta(p.D, d->rope_base, theta);
-  // Branch q/k rotated once at their semantic positions (sem_pos of the
-  // branch nodes); every key tile of a query tile reuses the rotated copy.
-  cudaError_t e = launch_rope2(p.dtype, q_br, q_rot, p.Hq, k_br, k_rot, p.Hkv, sem_pos + p.T_tot,
-                               p.R, p.D, theta, st);
-  if (e != cudaSuccess) return cuda_status(e);
+  cudaError_t e;
   if (p.dtype == SPECOPD_F32) {
+    // Branch q/k rotated once at their semantic positions (sem_pos of the
+    // branch nodes); every key block of a row reuses the rotated copy.
+    void* q_rot = ws + L.q_off;
+    void* k_rot = ws + L.k_off;
+    e = launch_rope2(p.dtype, q_br, q_rot, p.Hq, k_br, k_rot, p.Hkv, sem_pos + p.T_tot, p.R, p.D,
+                     theta, st);
+    if (e != cudaSuccess) return cuda_status(e);
     e = launch_attn_simt_f32(p, (const float*)q_rot, (const float*)k_rot, (const float*)v_br,
                              (const float*)k_tr, (const float*)v_tr, cu_trunk, anchors,
-                             (float*)out, lse, st);
+                             (float*)out, lse, st, false);
   } else {
-    e = launch_attn_sm100(p, q_rot, k_rot, v_br, k_tr, v_tr, cu_trunk, anchors, out, lse,
-                          ws + L.tail_off, L.total - L.tail_off, st);
+    e = launch_attn_sm100(p, q_br, k_br, v_br, k_tr, v_tr, cu_trunk, anchors, sem_pos + p.T_tot,
+                          theta, out, lse, ws + L.tail_off, L.total - L.tail_off, st, false);
+  }
+  return cuda_status(e);
+}
+
+size_t specopd_trunk_prefill_workspace_size(const specopd_attn_desc* d,
+                                            const int32_t* cu_trunk_host) {
+  if (!d) return 0;
+  CuTrunk cu;
+  if (read_cu(d->S, cu_trunk_host, cu) != SPECOPD_OK) return 0;
+  AttnProblem p;
+  if (attn_problem(d, cu, p) != SPECOPD_OK) return 0;
+  return attn_ws_layout(p, true).total;
+}
+
+specopd_status specopd_trunk_prefill(const specopd_attn_desc* d, const void* q_tr, void* k_tr,
+                                     const void* v_tr, const int32_t* cu_trunk,
+                                     const int32_t* cu_trunk_host, void* out, float* lse,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  if (!d) return SPECOPD_ERR_INVALID_ARG;
+  CuTrunk cu;
+  specopd_status s = read_cu(d->S, cu_trunk_host, cu);
+  if (s != SPECOPD_OK) return s;
+  AttnProblem p;
+  s = attn_problem(d, cu, p);
+  if (s != SPECOPD_OK) return s;
+  if (!q_tr || !k_tr || !v_tr || !cu_trunk || !out) return SPECOPD_ERR_INVALID_ARG;
+  const AttnWs L = attn_ws_layout(p, true);
+  if (!workspace || ws_bytes < L.total) return SPECOPD_ERR_WORKSPACE;
+  if (p.dtype == SPECOPD_BF16) {
+    if (!aligned16(q_tr) || !aligned16(k_tr) || !aligned16(v_tr) || !aligned16(out) ||
+        !aligned16(workspace))
+      return SPECOPD_ERR_UNSUPPORTED;
+  }
+  s = check_device();
+  if (s != SPECOPD_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  char* ws = reinterpret_cast<char*>(workspace);
+  double theta[128];
+  rope_theta(p.D, d->rope_base, theta);
+  // The K cache: trunk keys rotated in place at their positions.
+  cudaError_t e = launch_rope_trunk(p.dtype, k_tr, k_tr, cu_trunk, p.S, p.T_tot, p.Hkv, p.D,
+                                    theta, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (p.dtype == SPECOPD_F32) {
+    void* q_rot = ws + L.q_off;
+    e = launch_rope_trunk(p.dtype, q_tr, q_rot, cu_trunk, p.S, p.T_tot, p.Hq, p.D, theta, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = launch_attn_simt_f32(p, (const float*)q_rot, nullptr, nullptr, (const float*)k_tr,
+                             (const float*)v_tr, cu_trunk, nullptr, (float*)out, lse, st, true);
+  } else {
+    e = launch_attn_sm100(p, q_tr, k_tr, v_tr, k_tr, v_tr, cu_trunk, nullptr, nullptr, theta, out,
+                          lse, ws + L.tail_off, L.total - L.tail_off, st, true);
   }
   return cuda_status(e);
 }
@@ -248,21 +341,26 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* d, const void* z_target,
                               const int32_t* target_row, const void* z_draft, float* a,
                               float* prefix, float* loss, double* numer, void* grad_draft,
                               void* workspace, size_t ws_bytes, void* stream) {
-  TVProblem p;
-  specopd_status s = tv_problem(d, p);
+  return e2e_tv_checked(d, z_target, target_row, z_draft, a, prefix, loss, numer, grad_draft,
+                        workspace, ws_bytes, stream, false);
+}
+
+specopd_status specopd_e2e_tv_finalize(const double* numer_sum, int64_t norm_count,
+                                       float* loss, double* loss64, void* stream) {
+  if (!numer_sum || !loss || norm_count <= 0) return SPECOPD_ERR_INVALID_ARG;
+  specopd_status s = check_device();
   if (s != SPECOPD_OK) return s;
-  if (!z_target || !z_draft || !a || !prefix || !loss) return SPECOPD_ERR_INVALID_ARG;
-  if (p.compute_grad && !grad_draft) return SPECOPD_ERR_INVALID_ARG;
-  if (!target_row && p.rows_target < p.N) return SPECOPD_ERR_INVALID_ARG;
-  if (!workspace || ws_bytes < tv_workspace(p)) return SPECOPD_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return SPECOPD_ERR_UNSUPPORTED;
-  s = check_device();
+  return cuda_status(launch_tv_finalize(numer_sum, (double)norm_count, loss, loss64,
+                                        as_stream(stream)));
+}
+
+specopd_status specopd_debug_fault_injection(int64_t withhold_position,
+                                             uint64_t branch_wait_limit_ns) {
+  if (withhold_position < -1) return SPECOPD_ERR_INVALID_ARG;
+  specopd_status s = check_device();
   if (s != SPECOPD_OK) return s;
-  cudaError_t e = launch_e2e_tv(p, z_target, target_row, z_draft, a, prefix, loss, numer,
-                                p.compute_grad ? grad_draft : nullptr, workspace, ws_bytes,
-                                as_stream(stream));
-  if (e == cudaErrorInvalidConfiguration) { cudaGetLastError(); return SPECOPD_ERR_UNSUPPORTED; }
-  return cuda_status(e);
+  const FaultInject f = {(long long)withhold_position, (unsigned long long)branch_wait_limit_ns};
+  return cuda_status(cudaMemcpyToSymbol(specopd::g_inject, &f, sizeof(f)));
 }
 
 }  // extern "C"

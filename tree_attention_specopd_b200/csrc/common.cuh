@@ -26,6 +26,17 @@ __device__ unsigned int g_status = 0u;
 // Upper bound of every bounded wait (ns).  Normal waits last microseconds.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+// Host-driven fault injection for tests (specopd_debug_fault_injection):
+// off unless a test sets it.  withhold_position >= 0 makes the E2E-TV
+// scorer of that supervised position skip publishing its overlap, so the
+// other positions of its branch wait for it in vain; branch_wait_ns, when
+// nonzero, replaces kWaitLimitNs for those branch waits only.
+struct FaultInject {
+  long long withhold_position;
+  unsigned long long branch_wait_ns;
+};
+__device__ FaultInject g_inject = {-1ll, 0ull};
+
 __device__ __forceinline__ void set_status(unsigned bits) { atomicOr(&g_status, bits); }
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
@@ -82,6 +93,21 @@ __device__ __forceinline__ bool wait_flag_geq(const unsigned* flag, unsigned wan
     __nanosleep(64);
     if (ld_acquire_gpu(flag) >= want) return true;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(SPECOPD_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Same, with an explicit limit (ns).
+__device__ __forceinline__ bool wait_flag_geq_limit(const unsigned* flag, unsigned want,
+                                                    unsigned long long limit_ns) {
+  if (ld_acquire_gpu(flag) >= want) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) >= want) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_status(SPECOPD_DEV_TIMEOUT);
       return false;
     }

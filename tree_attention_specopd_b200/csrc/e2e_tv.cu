@@ -714,6 +714,58 @@ cudaError_t launch_row(const TVProblem& p, bool aligned, const void* z_target,
 
 }  // namespace
 
+// loss = 1 - numer_sum / norm (distributed normalisation, one thread).
+__global__ void tv_finalize_kernel(const double* numer_sum, double norm, float* loss,
+                                   double* loss64) {
+  const double l = 1.0 - numer_sum[0] / norm;
+  loss[0] = (float)l;
+  if (loss64) loss64[0] = l;
+}
+
+cudaError_t launch_tv_finalize(const double* numer_sum, double norm, float* loss, double* loss64,
+                               cudaStream_t st) {
+  tv_finalize_kernel<<<1, 1, 0, st>>>(numer_sum, norm, loss, loss64);
+  return cudaGetLastError();
+}
+
+namespace {
+
+// Rows and pointers that the vector and bulk-copy paths of the whole-row
+// schedule need: 16-byte aligned bases and row strides.
+bool rows_aligned(const TVProblem& p, const void* z_target, const void* z_draft, const void* grad) {
+  const int es = elt_size(p.logit_dtype);
+  const int gs = elt_size(p.grad_dtype);
+  const bool cg = p.compute_grad && grad != nullptr;
+  return ((uintptr_t)z_target % 16 == 0) && ((uintptr_t)z_draft % 16 == 0) &&
+         (!cg || (uintptr_t)grad % 16 == 0) && ((size_t)p.V * es % 16 == 0) &&
+         (!cg || (size_t)p.V * gs % 16 == 0);
+}
+
+// Whether the whole-row schedule runs this problem (one CTA per SM, rounds
+// of whole branches).
+bool row_applies(const TVProblem& p) {
+  void* fn = pick_row_kernel(p.logit_dtype, p.grad_dtype);
+  const size_t smem = ((sizeof(tvrow::Shared) + 127) / 128) * 128 +
+                      (size_t)tvrow::kStages * 2 * tvrow::kChunkBytes;
+  int dev = 0, per_sm = 0, nsm = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, tvrow::kThreads, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  return p.W <= (long long)std::min(per_sm, 1) * nsm;
+}
+
+}  // namespace
+
+size_t tv_workspace_for_call(const TVProblem& p, const void* z_target, const void* z_draft,
+                             const void* grad) {
+  if (rows_aligned(p, z_target, z_draft, grad) && row_applies(p)) return tvrow::row_layout(p).total;
+  return tv_workspace(p);
+}
+
 cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_t* target_row,
                           const void* z_draft, float* a, float* prefix, float* loss, double* numer,
                           void* grad, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -721,10 +773,7 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
   const int es = elt_size(p.logit_dtype);
   const int gs = elt_size(p.grad_dtype);
   {
-    const bool cg = p.compute_grad && grad != nullptr;
-    const bool aligned = ((uintptr_t)z_target % 16 == 0) && ((uintptr_t)z_draft % 16 == 0) &&
-                         (!cg || (uintptr_t)grad % 16 == 0) && ((size_t)p.V * es % 16 == 0) &&
-                         (!cg || (size_t)p.V * gs % 16 == 0);
+    const bool aligned = rows_aligned(p, z_target, z_draft, grad);
     const cudaError_t e = launch_row(p, aligned, z_target, target_row, z_draft, a, prefix, loss,
                                      numer, grad, ws, ws_bytes, stream);
     if (e != cudaErrorNotSupported) return e;

@@ -59,15 +59,17 @@ extern "C" specopd_status specopd_e2e_tv_noalloc(const specopd_tv_desc* desc,
                                                   float* loss, double* numer, void* grad_draft,
                                                   void* stream) {
   if (!desc) return SPECOPD_ERR_INVALID_ARG;
-  const size_t need = specopd_e2e_tv_workspace_size(desc);
-  if (need == 0) return SPECOPD_ERR_INVALID_ARG;  // the descriptor itself is invalid
-  if (need > specopd::kTVStaticScratchBytes) return SPECOPD_ERR_WORKSPACE;
+  if (specopd_e2e_tv_workspace_size(desc) == 0) return SPECOPD_ERR_INVALID_ARG;  // invalid descriptor
   void* scratch = nullptr;
   const cudaError_t e = specopd::tv_static_scratch(&scratch);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return SPECOPD_ERR_CUDA;
   }
-  return specopd_e2e_tv(desc, z_target, target_row, z_draft, a, prefix, loss, numer, grad_draft,
-                        scratch, specopd::kTVStaticScratchBytes, stream);
+  // The size limit applies to the scratch of the schedule this call runs:
+  // the whole-row schedule needs a few bytes per position, the slice
+  // fallback a few hundred.  Beyond the array: SPECOPD_ERR_WORKSPACE, before
+  // anything is launched.
+  return e2e_tv_checked(desc, z_target, target_row, z_draft, a, prefix, loss, numer, grad_draft,
+                        scratch, specopd::kTVStaticScratchBytes, stream, true);
 }

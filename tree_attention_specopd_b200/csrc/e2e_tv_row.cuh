@@ -202,6 +202,8 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       };
       const Tin *rt_prev = zt, *rd_prev = zd;
       for (int k = 0; k <= ntask && live; ++k) {
+        // Another warp's wait ran out (abort): issue nothing more.
+        if (__ldcg(&A.ctl[2]) != 0u) break;
         const bool hasA = k < ntask, hasC = grad && k > 0;
         const Tin *rt = zt, *rd = zd;
         if (hasA) {
@@ -219,6 +221,12 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
         rt_prev = rt;
         rd_prev = rd;
       }
+      // No copy may still be landing when this warp -- the last user of the
+      // CTA's shared memory that can start one -- returns: wait (bounded)
+      // for the last phase issued into every stage.  In a normal run the
+      // consumers have waited for each already and these return at once.
+      for (unsigned j = (q > (unsigned)kStages ? q - (unsigned)kStages : 0u); j < q; ++j)
+        mbar_wait(&sh.full[j % kStages], (j / kStages) & 1u);
     }
     return;
   }
@@ -234,9 +242,10 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       const int b = n / W, i = n % W;
       const bool owner = (i == 0);  // writes the branch's overlaps and prefix products
       int last = 0;
+      int ok_branch = 0;
       if (lane == 0) {
         // publish (a_n, s_n) once the 24 consumer warps' partials are in
-        bool in = mbar_wait(&sh.bdone, (unsigned)(k & 1));
+        const bool in = mbar_wait(&sh.bdone, (unsigned)(k & 1));
         float2 v = make_float2(qnan, qnan);
         if (in) {
           v = make_float2(0.f, 0.f);
@@ -247,18 +256,31 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
         } else {
           atomicExch(&A.ctl[2], 1u);
         }
-        A.part[n] = v;
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&A.br_cnt[b]) : "memory");
+        if ((long long)n != g_inject.withhold_position) {  // test hook: off by default
+          A.part[n] = v;
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&A.br_cnt[b]) : "memory");
+        }
         if (grad || owner) {
-          bool ok = in && __ldcg(&A.ctl[2]) == 0u;
-          if (ok) ok = wait_flag_geq(&A.br_cnt[b], (unsigned)W);
-          if (!ok) atomicExch(&A.ctl[2], 1u);
-          float s_own = qnan;
-          for (int j = 0; j < W; ++j) {
-            const float2 u = __ldcg(&A.part[(size_t)b * W + j]);
-            sh.sa[j] = ok ? u.x : qnan;
-            if (j == i) s_own = ok ? u.y : qnan;
-          }
+          // A branch wait that runs out makes this task's outputs NaN; it
+          // does not abort the copy ring (the other tasks go on).
+          const unsigned long long lim =
+              g_inject.branch_wait_ns ? g_inject.branch_wait_ns : kWaitLimitNs;
+          ok_branch = (in && __ldcg(&A.ctl[2]) == 0u &&
+                       wait_flag_geq_limit(&A.br_cnt[b], (unsigned)W, lim)) ? 1 : 0;
+        }
+      }
+      // The branch's W overlaps, one load per lane, each lane ordered after
+      // its own acquire of the (complete) counter.
+      ok_branch = __shfl_sync(0xffffffffu, ok_branch, 0);
+      if (grad || owner) {
+        if (ok_branch) ld_acquire_gpu(&A.br_cnt[b]);
+        for (int j = lane; j < W; j += 32)
+          sh.sa[j] = ok_branch ? __ldcg(&A.part[(size_t)b * W + j]).x : qnan;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        if (grad || owner) {
+          const float s_own = ok_branch ? __ldcg(&A.part[n]).y : qnan;
           // g_n = -(1/norm) P_{i-1} S_i, with no division by any overlap
           float P = 1.f;
           for (int j = 0; j < i; ++j) P *= sh.sa[j];

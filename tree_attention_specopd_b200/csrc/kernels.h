@@ -29,6 +29,11 @@ cudaError_t launch_tree_build(const CuTrunk& cu, const int32_t* anchors, int B, 
 // theta: host array of D/2 frequencies base^(-2k/D) in double precision.
 cudaError_t launch_rope(specopd_dtype dt, const void* x, void* y, const int32_t* pos, int n, int H,
                         int D, const double* theta_host, cudaStream_t st);
+// Trunk rows rotated at their position within their sequence (row t of
+// sequence s sits at t - cu[s]); cu_trunk is the device copy.
+cudaError_t launch_rope_trunk(specopd_dtype dt, const void* x, void* y, const int32_t* cu_trunk,
+                              int S, int n, int H, int D, const double* theta_host,
+                              cudaStream_t st);
 // Two tensors (H0 and H1 heads) rotated at the same positions in one launch.
 cudaError_t launch_rope2(specopd_dtype dt, const void* x0, void* y0, int H0, const void* x1,
                          void* y1, int H1, const int32_t* pos, int n, int D,
@@ -40,17 +45,27 @@ struct AttnProblem {
   float scale;  // softmax scale
   specopd_dtype dtype;
 };
+// prefill: q_rot is the rotated trunk queries [T_tot, Hq, D] and every trunk
+// row attends causally within its sequence (k_rot, v_br, anchors unused).
 cudaError_t launch_attn_simt_f32(const AttnProblem& p, const float* q_rot, const float* k_rot,
                                  const float* v_br, const float* k_tr, const float* v_tr,
                                  const int32_t* cu_trunk, const int32_t* anchors, float* out,
-                                 float* lse, cudaStream_t st);
+                                 float* lse, cudaStream_t st, bool prefill);
 
 // ---- tree attention, tcgen05/TMEM/TMA (bf16 workloads)
-size_t attn_sm100_workspace(const AttnProblem& p);
-cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_rot, const void* k_rot,
+size_t attn_sm100_workspace(const AttnProblem& p, bool prefill);
+// q_br / k_br are NOT rotated: the kernel rotates them at pos_br (the
+// semantic positions of the branch rows) with frequencies theta[D/2].
+// prefill: q_br is the trunk queries [T_tot, Hq, D] (rotated in the kernel at
+// their positions within their sequence), k_tr the rotated K cache, and the
+// output covers every trunk row (causal within each sequence); k_br, v_br,
+// anchors and pos_br are unused.
+cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_br, const void* k_br,
                               const void* v_br, const void* k_tr, const void* v_tr,
-                              const int32_t* cu_trunk, const int32_t* anchors, void* out,
-                              float* lse, void* ws, size_t ws_bytes, cudaStream_t st);
+                              const int32_t* cu_trunk, const int32_t* anchors,
+                              const int32_t* pos_br, const double* theta, void* out,
+                              float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
+                              bool prefill);
 
 // ---- E2E-TV
 struct TVProblem {
@@ -60,7 +75,13 @@ struct TVProblem {
   double norm_count;
 };
 size_t tv_workspace(const TVProblem& p);
+// Workspace bytes of the schedule launch_e2e_tv picks for these pointers on
+// the current device (at most tv_workspace(p)).
+size_t tv_workspace_for_call(const TVProblem& p, const void* z_target, const void* z_draft,
+                             const void* grad);
 int tv_slice_count(const TVProblem& p);
+cudaError_t launch_tv_finalize(const double* numer_sum, double norm, float* loss, double* loss64,
+                               cudaStream_t st);
 cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_t* target_row,
                           const void* z_draft, float* a, float* prefix, float* loss, double* numer,
                           void* grad, void* ws, size_t ws_bytes, cudaStream_t st);

@@ -35,9 +35,23 @@ constexpr int kRopeHeadGroup = 8;  // heads per thread: loads batched ahead of t
 // is reduced and its sine/cosine evaluated once per group, and the 16 loads
 // of the group are issued before any store (the tensor may be rotated in
 // place, so loads and stores of one head cannot be reordered by the compiler).
+// Position of row t: pos[t], or, with pos == NULL, its index within its
+// trunk sequence (t - cu[s] for cu[s] <= t < cu[s+1]; cu has S + 1 entries).
+__device__ __forceinline__ int row_position(const int32_t* __restrict__ pos,
+                                            const int32_t* __restrict__ cu, int S, long long t) {
+  if (pos) return pos[t];
+  int lo = 0, hi = S - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return (int)(t - cu[lo]);
+}
+
 template <typename T>
 __global__ void rope_kernel(const RopeJob j0, const RopeJob j1, const int32_t* __restrict__ pos,
-                            int n, int D, const RopeTheta th) {
+                            const int32_t* __restrict__ cu, int S, int n, int D,
+                            const RopeTheta th) {
   const int half = D >> 1;
   const int g0 = (j0.H + kRopeHeadGroup - 1) / kRopeHeadGroup;
   const int g1 = (j1.H + kRopeHeadGroup - 1) / kRopeHeadGroup;
@@ -55,7 +69,7 @@ __global__ void rope_kernel(const RopeJob j0, const RopeJob j1, const int32_t* _
     const RopeJob& J = first ? j0 : j1;
     const int hb = (first ? grp : grp - g0) * kRopeHeadGroup;
     const int nh = min(kRopeHeadGroup, J.H - hb);
-    const double ang = (double)pos[t] * th.theta[k];
+    const double ang = (double)row_position(pos, cu, S, t) * th.theta[k];
     const double red = ang - two_pi * rint(ang * inv_two_pi);
     float sn, cs;
     sincosf((float)red, &sn, &cs);
@@ -79,9 +93,10 @@ __global__ void rope_kernel(const RopeJob j0, const RopeJob j1, const int32_t* _
   }
 }
 
-cudaError_t launch_rope2(specopd_dtype dt, const void* x0, void* y0, int H0, const void* x1,
-                         void* y1, int H1, const int32_t* pos, int n, int D,
-                         const double* theta_host, cudaStream_t st) {
+namespace {
+cudaError_t rope_launch(specopd_dtype dt, const void* x0, void* y0, int H0, const void* x1,
+                        void* y1, int H1, const int32_t* pos, const int32_t* cu, int S, int n,
+                        int D, const double* theta_host, cudaStream_t st) {
   RopeTheta th;
   for (int k = 0; k < D / 2; ++k) th.theta[k] = theta_host[k];
   const RopeJob j0{x0, y0, H0};
@@ -94,10 +109,23 @@ cudaError_t launch_rope2(specopd_dtype dt, const void* x0, void* y0, int H0, con
   long long blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 64) blocks = 148 * 64;
   if (dt == SPECOPD_F32)
-    rope_kernel<float><<<(int)blocks, threads, 0, st>>>(j0, j1, pos, n, D, th);
+    rope_kernel<float><<<(int)blocks, threads, 0, st>>>(j0, j1, pos, cu, S, n, D, th);
   else
-    rope_kernel<__nv_bfloat16><<<(int)blocks, threads, 0, st>>>(j0, j1, pos, n, D, th);
+    rope_kernel<__nv_bfloat16><<<(int)blocks, threads, 0, st>>>(j0, j1, pos, cu, S, n, D, th);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_rope2(specopd_dtype dt, const void* x0, void* y0, int H0, const void* x1,
+                         void* y1, int H1, const int32_t* pos, int n, int D,
+                         const double* theta_host, cudaStream_t st) {
+  return rope_launch(dt, x0, y0, H0, x1, y1, H1, pos, nullptr, 0, n, D, theta_host, st);
+}
+
+cudaError_t launch_rope_trunk(specopd_dtype dt, const void* x, void* y, const int32_t* cu_trunk,
+                              int S, int n, int H, int D, const double* theta_host,
+                              cudaStream_t st) {
+  return rope_launch(dt, x, y, H, nullptr, nullptr, 0, nullptr, cu_trunk, S, n, D, theta_host, st);
 }
 
 cudaError_t launch_rope(specopd_dtype dt, const void* x, void* y, const int32_t* pos, int n, int H,

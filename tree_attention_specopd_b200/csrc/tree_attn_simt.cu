@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(1024) attn_simt_kernel(
     const AttnProblem p, const float* __restrict__ q_rot, const float* __restrict__ k_rot,
     const float* __restrict__ v_br, const float* __restrict__ k_tr,
     const float* __restrict__ v_tr, const int32_t* __restrict__ cu_trunk,
-    const int32_t* __restrict__ anchors, float* __restrict__ out, float* __restrict__ lse) {
+    const int32_t* __restrict__ anchors, float* __restrict__ out, float* __restrict__ lse,
+    int prefill) {
   constexpr int DPL = D / 32;  // output dims per lane
   extern __shared__ __align__(16) float simt_smem[];
   const int r = blockIdx.x;
@@ -39,11 +40,25 @@ __global__ void __launch_bounds__(1024) attn_simt_kernel(
   float* sq = simt_smem + warp * (D + 32);  // this head's scaled q
   float* sp = sq + D;                       // p of the current key block
   const int h = hk * p.G + warp;
+  // Branch row r = (s, b, i): trunk keys 0..a of sequence s, then branch
+  // nodes 1..i.  Trunk prefill (row r = a trunk row): the keys of its own
+  // sequence up to itself, i.e. a = its position, no branch keys.
   const int Wm1 = p.W - 1;
-  const int bid = r / Wm1;
-  const int i = r % Wm1 + 1;
-  const int s = bid / p.B;
-  const int a = anchors[bid];
+  int bid = 0, i = 0, s = 0, a = 0;
+  if (prefill) {
+    int lo = 0, hi = p.S - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cu_trunk[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    s = lo;
+    a = r - cu_trunk[s];
+  } else {
+    bid = r / Wm1;
+    i = r % Wm1 + 1;
+    s = bid / p.B;
+    a = anchors[bid];
+  }
   const int t0 = cu_trunk[s];
   const int Ts = cu_trunk[s + 1] - t0;
   float* o = out + ((long long)r * p.Hq + h) * D;
@@ -111,18 +126,19 @@ __global__ void __launch_bounds__(1024) attn_simt_kernel(
 cudaError_t launch_attn_simt_f32(const AttnProblem& p, const float* q_rot, const float* k_rot,
                                  const float* v_br, const float* k_tr, const float* v_tr,
                                  const int32_t* cu_trunk, const int32_t* anchors, float* out,
-                                 float* lse, cudaStream_t st) {
-  if (p.R == 0) return cudaSuccess;
+                                 float* lse, cudaStream_t st, bool prefill) {
+  const int nq = prefill ? p.T_tot : p.R;
+  if (nq == 0) return cudaSuccess;
   if (p.G < 1 || p.G > 32) return cudaErrorInvalidValue;
-  dim3 grid(p.R, p.Hkv);
+  dim3 grid(nq, p.Hkv);
   dim3 block(32 * p.G);
   const size_t smem = (size_t)p.G * (p.D + 32) * sizeof(float);
   if (p.D == 64)
     attn_simt_kernel<64><<<grid, block, smem, st>>>(p, q_rot, k_rot, v_br, k_tr, v_tr, cu_trunk,
-                                                    anchors, out, lse);
+                                                    anchors, out, lse, prefill ? 1 : 0);
   else if (p.D == 128)
     attn_simt_kernel<128><<<grid, block, smem, st>>>(p, q_rot, k_rot, v_br, k_tr, v_tr, cu_trunk,
-                                                     anchors, out, lse);
+                                                     anchors, out, lse, prefill ? 1 : 0);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

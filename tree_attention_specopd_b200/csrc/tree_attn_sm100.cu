@@ -24,6 +24,11 @@
 //  * Two CTAs share an SM (TMEM: 256 of the 512 columns each; shared memory
 //    under half), so one CTA's softmax overlaps the other's MMAs, and one
 //    CTA's prologue and epilogue overlap the other's main loop.
+//  * RoPE of the branch rows is fused: the query tile and the branch key
+//    tiles arrive unrotated by TMA, and the softmax warps rotate them in
+//    shared memory at each row's semantic position (review §3.2(a)) before
+//    the first MMA reads them; the branch key tiles come first in the key
+//    order of the leading chunk, so this happens in the prologue.
 //  * Per unit, warp 0 drives TMA (Q once, then 64-key K/V tiles in a 2-stage
 //    ring, 128-byte swizzle), warp 1 issues tcgen05.mma from one thread:
 //    S = Q K^T into TMEM (two S buffers, so QK^T of tile j+1 overlaps the
@@ -58,12 +63,16 @@ constexpr float kRescaleThreshold = 8.f;    // log2 units
 
 struct Params {
   int S, B, W, Hq, Hkv, G, R;
+  int prefill;         // 1: trunk prefill (query rows = trunk rows, causal within a sequence)
+  int T_tot;
   int RT;              // branch rows per query tile
   int ntile_per_seq, ntile;
   int nsplit, C;       // key chunks per (tile, kv head), keys per chunk (multiple of kBN)
   float scale_log2;    // softmax scale * log2(e)
   const int32_t* cu_trunk;
   const int32_t* anchors;
+  const int32_t* pos_br;  // semantic position of every branch row (sem_pos of the branch nodes)
+  double theta[64];       // RoPE frequencies base^(-2k/D), k < D/2 (double: angles reach ~3e4 rad)
   __nv_bfloat16* out;
   float* lse;
   float* part;         // split-KV partials
@@ -77,6 +86,7 @@ struct Hdr {
   uint64_t s_full[2], p_full[2];
   uint64_t o_done;   // one phase per P.V tile (used by the lazy rescale)
   uint64_t o_final;  // single phase: every MMA of the unit has completed
+  uint64_t rot_done; // single phase: Q and the branch key tiles are rotated (softmax warps)
   uint32_t tmem_base;
   int wmax[4];       // per-warp maxima of the tile's anchors
   int last;
@@ -210,6 +220,47 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// RoPE of one row held in shared memory as 128-byte swizzled lines (the
+// layout TMA writes with SWIZZLE_128B): pairs (d, d + D/2) for the pair
+// chunks c in [c0, c1), chunk c holding d = 8c .. 8c + 7.  For D = 128 the
+// two halves of the row are the same line of two 64-column boxes (same
+// swizzle), for D = 64 they are chunks c and c + 4 of one line.  The angle
+// pos * theta_d is formed and reduced to [-pi, pi] in double precision, as in
+// specopd_rope_apply, then evaluated in fp32; results are rounded to bf16.
+template <int D>
+__device__ __forceinline__ void rope_row_smem(uint8_t* lo_line, uint8_t* hi_line, int line, int pos,
+                                              const double* theta, int c0, int c1) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+  const int sw = line & 7;
+  for (int c = c0; c < c1; ++c) {
+    uint4* pa = reinterpret_cast<uint4*>(lo_line + ((c ^ sw) << 4));
+    uint4* pb = reinterpret_cast<uint4*>(hi_line + (((D == 128 ? c : c + 4) ^ sw) << 4));
+    const uint4 a = *pa, b = *pb;
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+    uint32_t ra[4], rb[4];
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+      float ya[2], yb[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const double ang = (double)pos * theta[8 * c + 2 * e2 + h];
+        const float red = (float)(ang - two_pi * rint(ang * inv_two_pi));
+        float sn, cs;
+        __sincosf(red, &sn, &cs);
+        const float xa = h ? bf16hi(wa[e2]) : bf16lo(wa[e2]);
+        const float xb = h ? bf16hi(wb[e2]) : bf16lo(wb[e2]);
+        ya[h] = xa * cs - xb * sn;
+        yb[h] = xb * cs + xa * sn;
+      }
+      ra[e2] = pack_bf16x2(ya[0], ya[1]);
+      rb[e2] = pack_bf16x2(yb[0], yb[1]);
+    }
+    *pa = make_uint4(ra[0], ra[1], ra[2], ra[3]);
+    *pb = make_uint4(rb[0], rb[1], rb[2], rb[3]);
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 template <int D>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
@@ -239,16 +290,36 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   // ---- work unit: (query tile, kv head, key chunk), chunk-major so that the
   // full leading chunks start first and the partial or empty trailing ones
   // fill in last; within a chunk, heavier tiles (larger anchors) first.
+  //
+  // Branch pass: a query tile is RT branch rows of one sequence s; its keys
+  // are trunk rows t0 + 0 .. t0 + a (t0 = start of s, a = the row's anchor)
+  // and its branch nodes.  Trunk prefill: a query tile is RT consecutive
+  // packed trunk rows (it may span a sequence boundary); its keys are the
+  // packed trunk rows t0 .. r, t0 = start of the sequence of the tile's
+  // first row, and row r sees the rows of its own sequence up to itself.
+  // In both cases row r sees the keys t0 + vlo_r .. t0 + vhi_r.
   const int u = blockIdx.x;
   const int per_c = P.ntile * P.Hkv;
   const int c = u / per_c;
   const int tile = P.ntile - 1 - (u % per_c) / P.Hkv;
   const int h = (u % per_c) % P.Hkv;
-  const int s = tile / P.ntile_per_seq;
   const int Wm1 = P.W - 1;
-  const int rows_seq = P.B * Wm1;
-  const int r0 = s * rows_seq + (tile % P.ntile_per_seq) * P.RT;
-  const int r1 = min(r0 + P.RT, (s + 1) * rows_seq);
+  int s, r0, r1;
+  if (P.prefill) {
+    r0 = tile * P.RT;
+    r1 = min(r0 + P.RT, P.T_tot);
+    int lo = 0, hi = P.S - 1;  // sequence of row r0: cu[s] <= r0 < cu[s+1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (P.cu_trunk[mid] <= r0) lo = mid; else hi = mid - 1;
+    }
+    s = lo;
+  } else {
+    s = tile / P.ntile_per_seq;
+    const int rows_seq = P.B * Wm1;
+    r0 = s * rows_seq + (tile % P.ntile_per_seq) * P.RT;
+    r1 = min(r0 + P.RT, (s + 1) * rows_seq);
+  }
   const int t0 = P.cu_trunk[s];
   const int Ts = P.cu_trunk[s + 1] - t0;
   const int G = P.G;
@@ -272,6 +343,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     mbar_init(&hdr->o_done, 1);
     mbar_init(&hdr->o_final, 1);
+    mbar_init(&hdr->rot_done, 128);
     hdr->abort = 0;
     fence_mbar_init();
     mbar_arrive_expect_tx(&hdr->q_full, (unsigned)(NH * MT * 128));
@@ -283,8 +355,12 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int r = r0 + warp * 32 + lane;
     int a = -1;
     if (r < r1) {
-      a = P.anchors[r / Wm1];
-      if (a < 0 || a >= Ts) a = -1;
+      if (P.prefill) {
+        a = r - t0;
+      } else {
+        a = P.anchors[r / Wm1];
+        if (a < 0 || a >= Ts) a = -1;
+      }
     }
     a = __reduce_max_sync(0xffffffffu, a);
     if (lane == 0) hdr->wmax[warp] = a;
@@ -326,8 +402,8 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     return;
   }
-  const int kb0 = (r0 / Wm1) * Wm1;  // first branch node the tile needs
-  const int nbt = (c == 0) ? (r1 - kb0 + kBN - 1) / kBN : 0;
+  const int kb0 = P.prefill ? 0 : (r0 / Wm1) * Wm1;  // first branch node the tile needs
+  const int nbt = (c == 0 && !P.prefill) ? (r1 - kb0 + kBN - 1) / kBN : 0;
   const int nk = nt + nbt;
   const uint32_t tS[2] = {tmem, tmem + kBN};
   const uint32_t tO = tmem + 2 * kBN;
@@ -338,7 +414,9 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // K tiles run kKStages - kVStages tiles ahead of V tiles: the QK^T that
       // frees a K slot completes before the P.V that frees the V slot of the
       // same tile, so a blocked V copy never holds back the next K copy.
-      auto row_of = [&](int j) { return j < nt ? t0 + k_begin + j * kBN : kb0 + (j - nt) * kBN; };
+      // Key order: the branch tiles (leading chunk only) first, so that the
+      // softmax warps can rotate them in the prologue, then the trunk tiles.
+      auto row_of = [&](int j) { return j < nbt ? kb0 + j * kBN : t0 + k_begin + (j - nbt) * kBN; };
       constexpr int kLead = kKStages - kVStages;
       for (int i = 0; i < nk + kLead && !hdr->abort; ++i) {
         if (i < nk) {
@@ -346,7 +424,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           if (j >= kKStages && !wait_or_abort(&hdr->k_empty[st], ((j / kKStages) - 1) & 1, hdr)) break;
           mbar_arrive_expect_tx(&hdr->k_full[st], NH * kKVHalf);
           for (int hh = 0; hh < NH; ++hh)
-            tma_load_3d(sK + (st * NH + hh) * kKVHalf, j < nt ? &tm_ktr : &tm_kbr, hh * 64, h,
+            tma_load_3d(sK + (st * NH + hh) * kKVHalf, j < nbt ? &tm_kbr : &tm_ktr, hh * 64, h,
                         row_of(j), &hdr->k_full[st]);
         }
         if (i >= kLead) {
@@ -354,7 +432,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           if (j >= kVStages && !wait_or_abort(&hdr->v_empty[st], ((j / kVStages) - 1) & 1, hdr)) break;
           mbar_arrive_expect_tx(&hdr->v_full[st], NH * kKVHalf);
           for (int hh = 0; hh < NH; ++hh)
-            tma_load_3d(sV + (st * NH + hh) * kKVHalf, j < nt ? &tm_vtr : &tm_vbr, hh * 64, h,
+            tma_load_3d(sV + (st * NH + hh) * kKVHalf, j < nbt ? &tm_vbr : &tm_vtr, hh * 64, h,
                         row_of(j), &hdr->v_full[st]);
         }
       }
@@ -384,7 +462,9 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_commit(&hdr->o_done);
         return true;
       };
-      bool ok = wait_or_abort(&hdr->q_full, 0, hdr);
+      // Q (and the leading branch key tiles) are rotated in shared memory
+      // by the softmax warps before the first MMA reads them.
+      bool ok = wait_or_abort(&hdr->rot_done, 0, hdr);
       tc_fence_after();
       for (int j = 0; j < nk && ok; ++j) {
         const int st = j % kKStages;
@@ -419,16 +499,49 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int lr = mrow / G, g = mrow % G;
     const int r = r0 + lr;
     const bool in_tile = (lr < P.RT) && (r < r1);
-    int a_r = -1, kfirst = 0;
+    int a_r = -1, kfirst = 0, vlo = 0, qpos = 0;
     bool bad = false;
     if (in_tile) {
-      const int bid = r / Wm1;
-      a_r = P.anchors[bid];
-      bad = (a_r < 0 || a_r >= Ts);
-      kfirst = bid * Wm1;
+      if (P.prefill) {
+        int sr = s;  // the row's own sequence (a tile spans few sequences)
+        while (sr + 1 < P.S && P.cu_trunk[sr + 1] <= r) ++sr;
+        vlo = P.cu_trunk[sr] - t0;
+        a_r = r - t0;
+        qpos = r - P.cu_trunk[sr];
+      } else {
+        const int bid = r / Wm1;
+        a_r = P.anchors[bid];
+        bad = (a_r < 0 || a_r >= Ts);
+        kfirst = bid * Wm1;
+        qpos = P.pos_br[r];
+      }
     }
     const bool live = in_tile && !bad;
     const float sl2 = P.scale_log2;
+    {
+      // ---- RoPE in shared memory: this thread's query row (TMEM lane =
+      // Q line), then half a line of each leading branch key tile.  The
+      // async proxy (tcgen05.mma) reads them after the fence and rot_done.
+      bool okr = warp_wait_or_abort(&hdr->q_full, 0, hdr);
+      if (okr && in_tile)
+        rope_row_smem<D>(sQ + mrow * 128, sQ + (D == 128 ? kQHalf : 0) + mrow * 128, mrow, qpos,
+                         P.theta, 0, D / 16);
+      const int t128 = tid - 64;  // 0..127
+      for (int j = 0; j < nbt; ++j) {
+        // branch tile j sits in K stage j (nbt <= 2 < kKStages), first use
+        okr = okr && warp_wait_or_abort(&hdr->k_full[j], 0, hdr);
+        const int line = t128 >> 1;
+        const int node = kb0 + j * kBN + line;
+        if (okr && node < P.R) {
+          uint8_t* base = sK + (j * NH) * kKVHalf + line * 128;
+          const int half = D / 32;  // pair chunks per thread
+          rope_row_smem<D>(base, base + (D == 128 ? kKVHalf : 0), line, P.pos_br[node], P.theta,
+                           (t128 & 1) * half, (t128 & 1) * half + half);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&hdr->rot_done);
+    }
     float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum
     uint32_t sv[kBN];
     // After a wait runs out the warp keeps stepping through the loop with its
@@ -449,11 +562,11 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       // visible columns of the tile: lo <= col <= hi
       int lo, hi;
-      if (j < nt) {
-        lo = 0;
-        hi = a_r - (k_begin + j * kBN);
+      if (j >= nbt) {
+        lo = vlo - (k_begin + (j - nbt) * kBN);
+        hi = a_r - (k_begin + (j - nbt) * kBN);
       } else {
-        const int node0 = kb0 + (j - nt) * kBN;
+        const int node0 = kb0 + j * kBN;
         lo = kfirst - node0;
         hi = r - node0;
       }
@@ -668,20 +781,28 @@ struct Plan {
 // (SMs x 2), the smallest nsplit whose units fill every slot once: finer
 // chunks add per-unit prologue, epilogue and merge work.  With one to eight
 // waves of pairs, two chunks halve the tail of the last wave.
-Plan make_plan(const AttnProblem& p, int num_sms) {
+Plan make_plan(const AttnProblem& p, int num_sms, bool prefill) {
   Plan pl;
   pl.RT = 128 / p.G;
-  const int rows_seq = p.B * (p.W - 1);
-  pl.ntile_per_seq = (rows_seq + pl.RT - 1) / pl.RT;
-  pl.ntile = pl.ntile_per_seq * p.S;
+  if (prefill) {
+    // Tiles of RT packed trunk rows; a tile's keys start at the first
+    // sequence it touches, so a key range is at most T_max + RT long.
+    pl.ntile_per_seq = 0;
+    pl.ntile = (p.T_tot + pl.RT - 1) / pl.RT;
+  } else {
+    const int rows_seq = p.B * (p.W - 1);
+    pl.ntile_per_seq = (rows_seq + pl.RT - 1) / pl.RT;
+    pl.ntile = pl.ntile_per_seq * p.S;
+  }
+  const int key_span = prefill ? p.T_max + pl.RT : p.T_max;
   const long long base = (long long)pl.ntile * p.Hkv;
   const long long slots = (long long)std::max(1, num_sms) * kCtasPerSm;
   long long want = base < slots ? (slots + base - 1) / base : (base < 8 * slots ? 2 : 1);
-  const int max_split = std::max(1, p.T_max / (4 * kBN));  // chunks of at least 4 key tiles
+  const int max_split = std::max(1, key_span / (4 * kBN));  // chunks of at least 4 key tiles
   const int best = (int)std::min<long long>(std::min<long long>(want, max_split), 64);
-  int C = (p.T_max + best - 1) / best;
+  int C = (key_span + best - 1) / best;
   C = (C + kBN - 1) / kBN * kBN;
-  pl.nsplit = (p.T_max + C - 1) / C;
+  pl.nsplit = (key_span + C - 1) / C;
   pl.C = C;
   pl.part_bytes = pl.nsplit > 1 ? (size_t)pl.ntile * p.Hkv * pl.nsplit * ((size_t)128 * p.D + 256) * 4 : 0;
   pl.cnt_bytes = (size_t)pl.ntile * p.Hkv * 4;
@@ -707,36 +828,44 @@ int sm_count() {
 }  // namespace
 }  // namespace sm100
 
-size_t attn_sm100_workspace(const AttnProblem& p) {
-  const sm100::Plan pl = sm100::make_plan(p, sm100::sm_count());
+size_t attn_sm100_workspace(const AttnProblem& p, bool prefill) {
+  const sm100::Plan pl = sm100::make_plan(p, sm100::sm_count(), prefill);
   return ((pl.part_bytes + 255) & ~size_t(255)) + pl.cnt_bytes;
 }
 
-cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_rot, const void* k_rot,
+cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_br, const void* k_br,
                               const void* v_br, const void* k_tr, const void* v_tr,
-                              const int32_t* cu_trunk, const int32_t* anchors, void* out,
-                              float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+                              const int32_t* cu_trunk, const int32_t* anchors,
+                              const int32_t* pos_br, const double* theta, void* out,
+                              float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
+                              bool prefill) {
   using namespace sm100;
-  if (p.R == 0) return cudaSuccess;
+  const int nq = prefill ? p.T_tot : p.R;  // query rows
+  if (nq == 0) return cudaSuccess;
   if (p.D != 64 && p.D != 128) return cudaErrorInvalidValue;
-  const Plan pl = make_plan(p, sm_count());
+  const Plan pl = make_plan(p, sm_count(), prefill);
   const size_t part_off = 0;
   const size_t cnt_off = (pl.part_bytes + 255) & ~size_t(255);
   if (ws_bytes < cnt_off + pl.cnt_bytes) return cudaErrorInvalidValue;
   CUtensorMap tq, tktr, tvtr, tkbr, tvbr;
-  if (!make_map(&tq, q_rot, p.D, p.Hq, p.R, p.G, pl.RT) ||
+  // Prefill has no branch keys: the branch maps repeat the trunk ones.
+  if (!make_map(&tq, q_br, p.D, p.Hq, nq, p.G, pl.RT) ||
       !make_map(&tktr, k_tr, p.D, p.Hkv, p.T_tot, 1, kBN) ||
       !make_map(&tvtr, v_tr, p.D, p.Hkv, p.T_tot, 1, kBN) ||
-      !make_map(&tkbr, k_rot, p.D, p.Hkv, p.R, 1, kBN) ||
-      !make_map(&tvbr, v_br, p.D, p.Hkv, p.R, 1, kBN))
+      !make_map(&tkbr, prefill ? k_tr : k_br, p.D, p.Hkv, prefill ? p.T_tot : p.R, 1, kBN) ||
+      !make_map(&tvbr, prefill ? v_tr : v_br, p.D, p.Hkv, prefill ? p.T_tot : p.R, 1, kBN))
     return cudaErrorInvalidValue;
   Params P;
   P.S = p.S; P.B = p.B; P.W = p.W; P.Hq = p.Hq; P.Hkv = p.Hkv; P.G = p.G; P.R = p.R;
+  P.prefill = prefill ? 1 : 0;
+  P.T_tot = p.T_tot;
   P.RT = pl.RT; P.ntile_per_seq = pl.ntile_per_seq; P.ntile = pl.ntile;
   P.nsplit = pl.nsplit; P.C = pl.C;
   P.scale_log2 = p.scale * 1.4426950408889634f;
   P.cu_trunk = cu_trunk;
   P.anchors = anchors;
+  P.pos_br = pos_br;
+  for (int k = 0; k < 64; ++k) P.theta[k] = k < p.D / 2 ? theta[k] : 0.0;
   P.out = reinterpret_cast<__nv_bfloat16*>(out);
   P.lse = lse;
   char* w = reinterpret_cast<char*>(ws);

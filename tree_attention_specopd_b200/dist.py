@@ -11,8 +11,10 @@ With torch.distributed (NCCL on GPUs, gloo on CPU):
   * global_count(): all-reduce of the per-rank position counts, done once
     per step before the E2E-TV call; the result is the norm_count of every
     rank's call, so every rank's gradient already carries the global 1/N.
-  * global_loss(): all-reduce of the per-rank prefix-product sums (the
-    `numer` output of specopd_e2e_tv) after the call; loss = 1 - sum / N.
+  * global_numer(): all-reduce of the per-rank prefix-product sums (the
+    `numer` output of specopd_e2e_tv) after the call;
+  * global_loss(): that sum, then the library's specopd_e2e_tv_finalize,
+    which writes loss = 1 - sum / N on the device.
 """
 
 from __future__ import annotations
@@ -39,11 +41,19 @@ def global_count(local_positions: int, group=None, device="cpu") -> int:
     return int(t.item())
 
 
-def global_loss(numer: torch.Tensor, count: int, group=None) -> torch.Tensor:
-    """loss = 1 - (sum over ranks of the prefix-product sums) / count.
-
-    `numer` is this rank's fp64 numerator (1 element); it is all-reduced in
-    place and the global loss is returned as a 1-element fp64 tensor."""
+def global_numer(numer: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum over ranks of the prefix-product sums, in place.  `numer` is this
+    rank's fp64 numerator (1 element, the `numer` output of specopd_e2e_tv)."""
     if dist.is_initialized() and dist.get_world_size(group) > 1:
         dist.all_reduce(numer, group=group)
-    return 1.0 - numer / float(count)
+    return numer
+
+
+def global_loss(numer: torch.Tensor, count: int, loss: torch.Tensor = None, group=None,
+                stream=None) -> torch.Tensor:
+    """loss = 1 - (sum over ranks of the prefix-product sums) / count, on the
+    device: the all-reduce of `numer` (in place, a CUDA tensor), then the
+    library's specopd_e2e_tv_finalize.  Returns the fp32 loss (1 element)."""
+    from . import api
+    global_numer(numer, group)
+    return api.specopd_e2e_tv_finalize(numer, count, loss=loss, stream=stream)
