@@ -6,8 +6,10 @@ One step = one pass of the whole path over one batch of synthetic input:
   specopd_e2e_tv      (overlaps, prefix products, loss, d loss / d draft logits)
 on the 8B-shaped workload (T=4096, B=64 anchors over the response half, W=8,
 32 q / 8 kv heads, head_dim 128, bf16; vocab 151,936, N = 512 positions).
-The trunk K cache is rotated once before timing (it belongs to the trunk
-prefill, which runs once per trunk).
+The trunk K cache comes from specopd_trunk_prefill (causal attention of the
+trunk with the K cache written rotated), run once before timing: the trunk is
+prefilled once and shared by all of its branches.  Its time is reported
+beside the step (`prefill`), not inside it.
 
 Metric: scored branch rows per second, R = B(W-1) rows per step and per GPU.
 Multi-GPU (torchrun): every rank scores its own batch of branches (weak
@@ -67,6 +69,16 @@ def attention_flops(cfg, anchors):
     keys = 0
     for a in anchors:
         keys += sum(int(a) + 1 + i for i in range(1, W))
+    return 4.0 * cfg.D * cfg.Hq * keys
+
+
+def prefill_flops(cfg, cu):
+    """Algorithmic FLOPs of the trunk prefill: every trunk row t (position p
+    in its sequence) and q head scores and mixes p + 1 keys, 4*D each."""
+    keys = 0
+    for s in range(len(cu) - 1):
+        T = cu[s + 1] - cu[s]
+        keys += T * (T + 1) // 2
     return 4.0 * cfg.D * cfg.Hq * keys
 
 
@@ -135,9 +147,20 @@ class Problem:
         self.score_row = torch.empty(self.N, dtype=i32, device=dev)
         api.specopd_tree_build(self.cu_host, self.anchors, B, W, self.parent, self.sem_pos,
                                self.score_row)
-        # trunk K cache, rotated once (trunk prefill)
-        api.specopd_rope_apply(self.k_tr, self.sem_pos[: self.T_tot].contiguous(), acfg.rope_base)
         self.desc = api.attn_desc(S, B, W, acfg.Hq, acfg.Hkv, acfg.D, acfg.dtype, acfg.rope_base)
+        # Trunk prefill: trunk queries (seeded, N(0,1)), the raw trunk keys
+        # kept for timing it again, the K cache rotated in place by the call.
+        gq = torch.Generator(device=dev)
+        gq.manual_seed(4321 + seed_offset)
+        self.q_tr = torch.randn((self.T_tot, acfg.Hq, acfg.D), generator=gq, device=dev).to(adt)
+        self.k_raw = self.k_tr.clone()
+        self.out_tr = torch.empty_like(self.q_tr)
+        self.pf_ws = torch.empty(max(api.specopd_trunk_prefill_workspace_size(self.desc,
+                                                                              self.cu_host), 256),
+                                 dtype=torch.uint8, device=dev)
+        api.specopd_trunk_prefill(self.desc, self.q_tr, self.k_tr, self.v_tr, self.cu_dev,
+                                  self.cu_host, out=self.out_tr, workspace=self.pf_ws)
+        self.pf_flops = prefill_flops(acfg, self.cu_host)
         ws = api.specopd_tree_attn_workspace_size(self.desc, self.cu_host)
         self.attn_ws = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.out = torch.empty_like(self.q_br)
@@ -198,7 +221,31 @@ class Problem:
             ev[2].record()
 
 
-KERNELS_PER_STEP = 4  # tree_build, rope(branch q and k), tree_attn, e2e_tv
+    def time_prefill(self, reps=5):
+        """Device time (ms) of one specopd_trunk_prefill, on a fresh copy of
+        the raw trunk keys each time (the call rotates them in place; the
+        copy is outside the timed region)."""
+        torch = self.torch
+        k = torch.empty_like(self.k_raw)
+        evs = []
+        for i in range(reps + 2):
+            k.copy_(self.k_raw)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            self.api.specopd_trunk_prefill(self.desc, self.q_tr, k, self.v_tr, self.cu_dev,
+                                           self.cu_host, out=self.out_tr, workspace=self.pf_ws)
+            e1.record()
+            if i >= 2:
+                evs.append((e0, e1))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+
+
+def kernels_per_step(acfg):
+    """Library kernels one step launches: tree_build, tree_attn (branch RoPE
+    fused for bf16; a separate RoPE launch for the fp32 SIMT path), e2e_tv."""
+    return 3 if acfg.dtype == "bf16" else 4
 
 
 def run_gpu(args):
@@ -279,6 +326,20 @@ def run_gpu(args):
     # ---- end-to-end through the public API with host buffers (the default
     # workload; the larger ones would copy tens of GB per step)
     e2e = e2e_measure(torch, api, pb, args, dev, world) if wl == WORKLOAD else None
+    pf_ms = pb.time_prefill() if rank == 0 else None
+
+    # ---- the other workloads, device-timed in the same run (one GPU)
+    extra = None
+    if world == 1 and wl == WORKLOAD and not args.no_extra_workloads:
+        figs = _Figures(pb)
+        del pb
+        torch.cuda.empty_cache()
+        extra = {}
+        for other in ("tiny", "long", "packed"):
+            extra[other] = measure_workload(torch, api, dev, other, max(3, min(args.steps, 10)),
+                                            args.warmup)
+            torch.cuda.empty_cache()
+        pb = figs
 
     if rank == 0:
         peaks = _peaks()
@@ -286,6 +347,7 @@ def run_gpu(args):
         value = pb.R * world / (ms_step / 1e3)
         tv_gbs = pb.tv_bytes / (tv_ms / 1e3) / 1e9
         attn_tflops = pb.flops / (attn_ms / 1e3) / 1e12
+        pf_tflops = pb.pf_flops / (pf_ms / 1e3) / 1e12 if pf_ms else None
         clocks = _clock_summary(clk_path, local)
         traffic = _ncu_traffic() if wl == WORKLOAD else None  # counters of the 8B launch
         # DRAM bytes actually moved per launch (ncu) over the live launch time:
@@ -326,11 +388,20 @@ def run_gpu(args):
                                    if pb.acfg.dtype == "bf16" else None,
                                    "algorithmic_flops_per_launch": pb.flops, "launch_ms": attn_ms,
                                    "peak_src": peaks["src"]},
+            "prefill": {"kernel": "tree_attn (trunk prefill mode) + K-cache RoPE",
+                        "note": "once per trunk, before the timed steps; not part of a step",
+                        "launch_ms": pf_ms, "algorithmic_flops_per_call": pb.pf_flops,
+                        "achieved": pf_tflops, "unit": "TFLOP/s",
+                        "peak": peaks["bf16_tflops"] if pb.acfg.dtype == "bf16" else None,
+                        "frac": pf_tflops / peaks["bf16_tflops"]
+                        if pf_tflops and pb.acfg.dtype == "bf16" else None},
             "loss": loss,
             "clocks": clocks,
             "e2e": e2e,
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "gpu_launches": kernels_per_step(pb.acfg) * args.steps,
         }
+        if extra is not None:
+            line["workloads"] = extra
         if e2e is None:
             line["e2e_note"] = "host-buffer end-to-end measured on the default 8B workload only"
         if not args.no_cpu_baseline:
@@ -341,9 +412,63 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+class _Figures:
+    """Per-step constants of a Problem (sizes, algorithmic work), kept after
+    its device buffers are released."""
+
+    def __init__(self, pb):
+        for k in ("acfg", "tcfg", "R", "N", "flops", "pf_flops", "tv_bytes"):
+            setattr(self, k, getattr(pb, k))
+
+
+def measure_workload(torch, api, dev, workload, steps, warmup):
+    """Device-timed step of another workload (CUDA events on the launching
+    stream, as for the main line): rows/s and both roofline fractions."""
+    pb = Problem(torch, api, dev, workload=workload)
+    for _ in range(warmup):
+        pb.step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(steps):
+        pb.step(evs[k])
+    e1.record()
+    torch.cuda.synchronize()
+    st = api.specopd_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x} on the {workload} workload")
+    peaks = _peaks()
+    ms = e0.elapsed_time(e1) / steps
+    attn_ms = sum(ev[0].elapsed_time(ev[1]) for ev in evs) / steps
+    tv_ms = sum(ev[1].elapsed_time(ev[2]) for ev in evs) / steps
+    pf_ms = pb.time_prefill(3)
+    bf = pb.acfg.dtype == "bf16"
+    tv_gbs = pb.tv_bytes / (tv_ms / 1e3) / 1e9
+    att = pb.flops / (attn_ms / 1e3) / 1e12
+    pft = pb.pf_flops / (pf_ms / 1e3) / 1e12
+    out = {"workload": WORKLOAD_NAMES[workload], "steps": steps, "warmup": warmup,
+           "ms_per_step": ms, "value": pb.R / (ms / 1e3), "unit": "rows/s",
+           "supervised_tokens_per_s": pb.N / (ms / 1e3),
+           "e2e_tv": {"launch_ms": tv_ms, "achieved_gbs": tv_gbs,
+                      "frac": tv_gbs / peaks["hbm_gbs"],
+                      "algorithmic_bytes_per_launch": pb.tv_bytes},
+           "tree_attn": {"launch_ms": attn_ms, "achieved_tflops": att,
+                         "frac": att / peaks["bf16_tflops"] if bf else None,
+                         "algorithmic_flops_per_launch": pb.flops},
+           "prefill": {"launch_ms": pf_ms, "achieved_tflops": pft,
+                       "frac": pft / peaks["bf16_tflops"] if bf else None},
+           "peak_src": peaks["src"],
+           "l2": "inputs larger than L2" if pb.tv_bytes / 2 > 126e6 else "inputs fit in L2"}
+    del pb
+    return out
+
+
 TV_SOURCES = (
     "tree_attention_specopd_b200/csrc/e2e_tv.cu",
     "tree_attention_specopd_b200/csrc/e2e_tv_row.cuh",
+    "tree_attention_specopd_b200/csrc/e2e_tv_cluster.cuh",
     "tree_attention_specopd_b200/csrc/common.cuh",
 )
 
@@ -412,28 +537,39 @@ def _ncu_traffic():
 
 
 def e2e_measure(torch, api, pb, args, dev, world):
-    """Same metric through the public API, host buffers: per step the branch
-    q/k/v, anchors and both logit batches are copied from pinned host memory,
-    and the loss is read back."""
+    """Same metric through the public API, host buffers.  Every step uploads
+    the step's inputs from pinned host memory -- branch q/k/v, anchors, the
+    draft logits, and the target rows straight into the packed table the
+    kernel reads through the score-row map (the W-1 branch rows of every
+    branch as one block, each anchor's trunk row on its own) -- runs the
+    step, and reads the step's results back: the fp32 gradient of the draft
+    logits, the attention output and the loss."""
     import torch.distributed as dist
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    T, R = pb.T_tot, pb.R
+    sr = pb.score_row.cpu().numpy()
+    W = pb.acfg.W
+    anchor_rows = [int(sr[b * W]) for b in range(pb.N // W)]  # position (b, 1): a trunk row
     h = {"q": pin(pb.q_br), "k": pin(pb.k_br), "v": pin(pb.v_br), "anc": pin(pb.anchors),
-         "zt": pin(pb.z_t[pb.score_row.long()]), "zd": pin(pb.z_d)}
-    zt_rows = torch.empty_like(pb.z_d)
-    sr_long = pb.score_row.long()
+         "zt_br": pin(pb.z_t[T: T + R]), "zt_anc": pin(pb.z_t[anchor_rows]), "zd": pin(pb.z_d)}
+    grad_h = torch.empty(pb.grad.shape, dtype=pb.grad.dtype).pin_memory()
+    out_h = torch.empty(pb.out.shape, dtype=pb.out.dtype).pin_memory()
     loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in h.values())
-    d2h = loss_h.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in (grad_h, out_h, loss_h))
 
     def one():
         pb.q_br.copy_(h["q"], non_blocking=True)
         pb.k_br.copy_(h["k"], non_blocking=True)
         pb.v_br.copy_(h["v"], non_blocking=True)
         pb.anchors.copy_(h["anc"], non_blocking=True)
-        zt_rows.copy_(h["zt"], non_blocking=True)
+        pb.z_t[T: T + R].copy_(h["zt_br"], non_blocking=True)
+        for b, row in enumerate(anchor_rows):
+            pb.z_t[row].copy_(h["zt_anc"][b], non_blocking=True)
         pb.z_d.copy_(h["zd"], non_blocking=True)
-        pb.z_t.index_copy_(0, sr_long, zt_rows)
         pb.step()
+        grad_h.copy_(pb.grad, non_blocking=True)
+        out_h.copy_(pb.out, non_blocking=True)
         loss_h.copy_(pb.loss, non_blocking=True)
 
     for _ in range(2):
@@ -454,8 +590,11 @@ def e2e_measure(torch, api, pb, args, dev, world):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
+    ok = bool(torch.isfinite(grad_h).all()) and abs(float(loss_h.item()) - float(pb.loss.item())) == 0
     return {"value": pb.R * world / (ms / 1e3), "unit": "rows/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "results_read_back": ["grad_draft (fp32)", "attention out", "loss"],
+            "read_back_finite": ok}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -537,6 +676,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="skip the device-timed secondary workloads of the default run")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOAD_NAMES),
                     help="synthetic configuration (default: the 8B-shaped one)")
     args = ap.parse_args()
