@@ -418,6 +418,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // softmax warps can rotate them in the prologue, then the trunk tiles.
       auto row_of = [&](int j) { return j < nbt ? kb0 + j * kBN : t0 + k_begin + (j - nbt) * kBN; };
       constexpr int kLead = kKStages - kVStages;
+      int nk_issued = 0, nv_issued = 0;
       for (int i = 0; i < nk + kLead && !hdr->abort; ++i) {
         if (i < nk) {
           const int j = i, st = j % kKStages;
@@ -426,6 +427,7 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int hh = 0; hh < NH; ++hh)
             tma_load_3d(sK + (st * NH + hh) * kKVHalf, j < nbt ? &tm_kbr : &tm_ktr, hh * 64, h,
                         row_of(j), &hdr->k_full[st]);
+          nk_issued = j + 1;
         }
         if (i >= kLead) {
           const int j = i - kLead, st = j % kVStages;
@@ -434,8 +436,18 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int hh = 0; hh < NH; ++hh)
             tma_load_3d(sV + (st * NH + hh) * kKVHalf, j < nbt ? &tm_vbr : &tm_vtr, hh * 64, h,
                         row_of(j), &hdr->v_full[st]);
+          nv_issued = j + 1;
         }
       }
+      // No copy may still be landing when the CTA's shared memory is
+      // released: wait (bounded, whatever the abort flag says) for the Q copy
+      // and the last phase issued into every K and V stage.  In a normal run
+      // the MMA warp has waited for each already and these return at once.
+      mbar_wait(&hdr->q_full, 0);
+      for (int j = max(0, nk_issued - kKStages); j < nk_issued; ++j)
+        mbar_wait(&hdr->k_full[j % kKStages], (j / kKStages) & 1);
+      for (int j = max(0, nv_issued - kVStages); j < nv_issued; ++j)
+        mbar_wait(&hdr->v_full[j % kVStages], (j / kVStages) & 1);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
@@ -638,7 +650,11 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
     }
     // ---- epilogue
-    const bool ok = warp_wait_or_abort(&hdr->o_final, 0, hdr) && !hdr->abort;
+    // o_final is committed by the MMA thread in every case, abort or not,
+    // and tracks every MMA it issued: wait for it (bounded) even after an
+    // abort, so no MMA still writes TMEM when it is read or deallocated.
+    const bool fin = __all_sync(0xffffffffu, mbar_wait(&hdr->o_final, 0));
+    const bool ok = fin && !hdr->abort;
     tc_fence_after();
     __syncwarp();
     const int hq = h * G + g;
