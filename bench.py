@@ -468,7 +468,6 @@ def measure_workload(torch, api, dev, workload, steps, warmup):
 TV_SOURCES = (
     "tree_attention_specopd_b200/csrc/e2e_tv.cu",
     "tree_attention_specopd_b200/csrc/e2e_tv_row.cuh",
-    "tree_attention_specopd_b200/csrc/e2e_tv_cluster.cuh",
     "tree_attention_specopd_b200/csrc/common.cuh",
 )
 
