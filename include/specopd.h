@@ -188,6 +188,8 @@ size_t specopd_tree_attn_workspace_size(const specopd_attn_desc* desc,
  * All tensors of one call share `dtype`.  R = S*B*(W-1); W = 1 is valid and
  * launches nothing.  An anchor outside its trunk sets
  * SPECOPD_DEV_ANCHOR_RANGE and that branch's rows are written as NaN.
+ * BF16 returns SPECOPD_ERR_UNSUPPORTED when floor(128 / (Hq/Hkv)) + W - 2 >
+ * 192 (a query tile's branch keys must fit three 64-key tiles).
  */
 specopd_status specopd_tree_attn(const specopd_attn_desc* desc,
                                  const void* q_br, const void* k_br,

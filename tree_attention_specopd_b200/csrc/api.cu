@@ -244,6 +244,10 @@ specopd_status specopd_tree_attn(const specopd_attn_desc* d, const void* q_br, c
   s = attn_problem(d, cu, p);
   if (s != SPECOPD_OK) return s;
   if (p.R == 0) return SPECOPD_OK;
+  // bf16: the branch keys of a query tile (its rows and the earlier nodes of
+  // its first branch, floor(128 / G) + W - 2 rows at most) are rotated in the
+  // kernel's K ring before the first MMA reads them: three 64-key tiles at most.
+  if (p.dtype == SPECOPD_BF16 && (128 / p.G + p.W - 2 + 63) / 64 > 3) return SPECOPD_ERR_UNSUPPORTED;
   if (!q_br || !k_br || !v_br || !k_tr || !v_tr || !cu_trunk || !anchors || !sem_pos || !out)
     return SPECOPD_ERR_INVALID_ARG;
   const AttnWs L = attn_ws_layout(p);

@@ -146,11 +146,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
       : "memory");
   return ok != 0;
 }
+// Same, with a suspend-time hint: the thread may sleep in the instruction
+// until the phase completes or about kSuspendNs have passed, so a waiting
+// warp takes no issue slots from the others.
+constexpr unsigned kSuspendNs = 1000000u;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity)) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       set_status(SPECOPD_DEV_TIMEOUT);
       return false;

@@ -62,6 +62,8 @@
 #include <mutex>
 #include <tuple>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 

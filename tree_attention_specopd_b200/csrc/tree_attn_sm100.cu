@@ -630,20 +630,24 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       }
       // p = 2^(s*scale*log2e - m); masked entries are -inf -> 0
+      // (packed fp32x2 arithmetic: one FFMA2 and one FADD2 per key pair; P
+      // as bf16 pairs overwrites sv in place, sv[e] having been read at step
+      // e / 2)
       const float nm = (m == -INFINITY) ? 0.f : -m;
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[kBN / 2];
+      const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(nm, nm);
+      float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int e = 0; e < kBN / 2; ++e) {
-        const float p0 = ex2_fast(__fmaf_rn(__uint_as_float(sv[2 * e]), sl2, nm));
-        const float p1 = ex2_fast(__fmaf_rn(__uint_as_float(sv[2 * e + 1]), sl2, nm));
-        rs4[e & 3] += p0 + p1;
-        pk[e] = pack_bf16x2(p0, p1);
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                                    sl2v, nmv);
+        const float2 p = make_float2(ex2_fast(x.x), ex2_fast(x.y));
+        rs2[e & 1] = __fadd2_rn(rs2[e & 1], p);
+        sv[e] = pack_bf16x2(p.x, p.y);
       }
-      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      l += (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
       if (!dead) {
         __syncwarp();
-        tmem_st32(tS[b] + lane_off, pk);  // P of the tile's kBN keys as bf16 pairs
+        tmem_st32(tS[b] + lane_off, sv);  // P of the tile's kBN keys as bf16 pairs
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&hdr->p_full[b]);
@@ -719,11 +723,20 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float mm = -INFINITY;
         for (int cc = 0; cc < nact; ++cc)
           mm = fmaxf(mm, __ldcg(pbase + cc * slot_floats + 128 * D + mrow));
-        float ll = 0.f;
+        // this chunk's own partial first: it is still in TMEM and registers
+        const float wown = (m == -INFINITY) ? 0.f : exp2f(m - mm);
+        float ll = wown * l;
         float acc[D];
 #pragma unroll
-        for (int e = 0; e < D; ++e) acc[e] = 0.f;
+        for (int q = 0; q < DC; ++q) {
+          uint32_t ov[32];
+          tmem_ld32(tO + lane_off + q * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) acc[q * 32 + e] = wown * __uint_as_float(ov[e]);
+        }
         for (int cc = 0; cc < nact; ++cc) {
+          if (cc == c) continue;  // added first, above
           const float* pc = pbase + cc * slot_floats;
           const float mc = __ldcg(pc + 128 * D + mrow);
           const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - mm);
