@@ -44,7 +44,7 @@ def test_workspace_sizes_are_host_only(lib):
     assert api.specopd_tree_attn_workspace_size(bad, [0, 4096]) == 0
     assert api.specopd_tree_attn_workspace_size(d, [1, 4096]) == 0  # cu[0] != 0
     assert api.specopd_e2e_tv_workspace_size(api.tv_desc(0, 8, 100, 10, "f32")) == 0
-    # vocabularies too large for the cluster-resident rows are unsupported
+    # vocabularies beyond the slice schedule's slice count are unsupported
     assert api.specopd_e2e_tv_workspace_size(api.tv_desc(1, 1, 10_000_000, 1, "f32")) == 0
 
 
@@ -59,3 +59,14 @@ def test_invalid_arguments_rejected_before_device(lib):
     # rope with odd D
     d = api.RopeDesc(7, 0, 10000.0)
     assert lib.specopd_rope_apply(ctypes.byref(d), None, None, 4, 1, None) == 1
+
+
+def test_bf16_branch_span_limit(lib):
+    # bf16 tree attention rotates a query tile's branch keys -- its
+    # floor(128 / G) rows plus up to W - 2 earlier nodes of its first branch --
+    # in three 64-key tiles; longer spans are refused before any device work.
+    cu = (ctypes.c_int32 * 2)(0, 4096)
+    fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    args = [fake] * 5 + [fake, cu, fake, fake, fake, None, fake, 1 << 20, None]
+    d = api.attn_desc(1, 4, 70, 8, 8, 128, "bf16")  # G = 1: 128 + 68 = 196 > 192
+    assert lib.specopd_tree_attn(ctypes.byref(d), *args) == 2  # SPECOPD_ERR_UNSUPPORTED
