@@ -54,6 +54,7 @@ struct Shared {
   uint64_t full[kStages], empty[kStages];
   uint64_t bdone;            // one phase per task: every consumer warp's pass-B partials are in
   uint64_t gfull;            // one phase per task: g_n and s_n are in
+  uint64_t lsebar;           // one phase per task: every consumer warp's pass-A record is in
   float4 red[2][kCWarps];    // per-warp (max, sum) of both rows after pass A, by task parity
   float2 redB[kCWarps];      // per-warp (a, s) partials after pass B
   float g, s_own;            // written by the scorer warp
@@ -109,9 +110,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
   return p;
 }
 
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 // (max, sum) pair of log2-domain statistics: combine two, branch-free.  An
 // empty side (max = -inf) contributes nothing; the result is symmetric in
 // the two operands bit for bit.
@@ -163,6 +161,7 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
     }
     mbar_init(&sh.bdone, kCWarps);
     mbar_init(&sh.gfull, 1);
+    mbar_init(&sh.lsebar, kCWarps);
     fence_mbar_init();
   }
   __syncthreads();
@@ -505,25 +504,38 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       if (hasA && i + kLag < nch) {
         const int c = i + kLag;
         if (c < nfull) chunkA(c, std::true_type{}); else chunkA(c, std::false_type{});
+        if (c == nch - 1) {
+          // Pass A of this warp is complete: its record of the row
+          // statistics goes in now, and the warp waits for the others'
+          // only after the C chunks that follow (the last kLag of pass C),
+          // so those absorb the warps' skew.
+          float sum_t = (at0.x + at0.y) + (at1.x + at1.y);
+          float sum_d = (ad0.x + ad0.y) + (ad1.x + ad1.y);
+          // -inf maximum: this thread saw no finite entry of that row, no mass
+          if (mt == -INFINITY) sum_t = 0.f;
+          if (md == -INFINITY) sum_d = 0.f;
+          warp_lse2_merge(mt, sum_t);
+          warp_lse2_merge(md, sum_d);
+          if (lane == 0) {
+            sh.red[k & 1][warp] = make_float4(mt, sum_t, md, sum_d);
+            mbar_arrive(&sh.lsebar);
+          }
+        }
       }
     }
     if (!hasA) break;  // the last phase held only the last gradient row
 
     // ------------------------------ lse of task k
-    float sum_t = (at0.x + at0.y) + (at1.x + at1.y);
-    float sum_d = (ad0.x + ad0.y) + (ad1.x + ad1.y);
-    // -inf maximum: this thread saw no finite entry of that row, no mass
-    if (mt == -INFINITY) sum_t = 0.f;
-    if (md == -INFINITY) sum_d = 0.f;
-    warp_lse2_merge(mt, sum_t);
-    warp_lse2_merge(md, sum_d);
-    if (lane == 0) sh.red[k & 1][warp] = make_float4(mt, sum_t, md, sum_d);
-    named_sync(1, kConsumers);
-    // Every warp combines the warp records itself (no second barrier).  The
-    // combination is symmetric in its two operands, so the butterfly leaves
-    // the same bits in every lane, and every warp computes the same L.  The
-    // records alternate between two buffers by task parity: a warp reaches
-    // the next write of this buffer only through the next task's barrier.
+    // Every warp waits for the 24 records (bounded), then combines them
+    // itself.  The combination is symmetric in its two operands, so the
+    // butterfly leaves the same bits in every lane, and every warp computes
+    // the same L.  The records alternate between two buffers by task parity:
+    // a warp writes this buffer again (task k + 2) only after waiting for
+    // task k + 1's records, which every warp writes after reading these.
+    if (!dead && !mbar_wait(&sh.lsebar, (unsigned)(k & 1))) {
+      dead = true;
+      atomicExch(&A.ctl[2], 1u);
+    }
     float2 L;
     {
       float4 v = lane < kCWarps ? sh.red[k & 1][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
