@@ -542,7 +542,15 @@ def e2e_measure(torch, api, pb, args, dev, world):
     kernel reads through the score-row map (the W-1 branch rows of every
     branch as one block, each anchor's trunk row on its own) -- runs the
     step, and reads the step's results back: the fp32 gradient of the draft
-    logits, the attention output and the loss."""
+    logits, the attention output and the loss.
+
+    Steps are pipelined over two sets of device buffers, as a training loop
+    would run them: while step i computes on one set, the copy streams
+    upload step i+1's inputs into the other and read step i-1's results
+    out of it.  Events order the three streams: a set's inputs are
+    overwritten only after the step that read them finished, and its outputs
+    only after they were copied out.  The timed region runs from before the
+    first upload to after the last read-back."""
     import torch.distributed as dist
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
     T, R = pb.T_tot, pb.R
@@ -551,47 +559,83 @@ def e2e_measure(torch, api, pb, args, dev, world):
     anchor_rows = [int(sr[b * W]) for b in range(pb.N // W)]  # position (b, 1): a trunk row
     h = {"q": pin(pb.q_br), "k": pin(pb.k_br), "v": pin(pb.v_br), "anc": pin(pb.anchors),
          "zt_br": pin(pb.z_t[T: T + R]), "zt_anc": pin(pb.z_t[anchor_rows]), "zd": pin(pb.z_d)}
-    grad_h = torch.empty(pb.grad.shape, dtype=pb.grad.dtype).pin_memory()
-    out_h = torch.empty(pb.out.shape, dtype=pb.out.dtype).pin_memory()
-    loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+    names = ("q_br", "k_br", "v_br", "anchors", "z_t", "z_d", "out", "grad", "loss")
+    sets = [{n: getattr(pb, n) for n in names},
+            {n: torch.empty_like(getattr(pb, n)) for n in names}]
+    outs = [{"grad": torch.empty(pb.grad.shape, dtype=pb.grad.dtype).pin_memory(),
+             "out": torch.empty(pb.out.shape, dtype=pb.out.dtype).pin_memory(),
+             "loss": torch.empty(1, dtype=torch.float32).pin_memory()} for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in h.values())
-    d2h = sum(t.numel() * t.element_size() for t in (grad_h, out_h, loss_h))
+    d2h = sum(t.numel() * t.element_size() for t in outs[0].values())
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    done = [None, None]     # compute of the set's last step finished
+    copied = [None, None]   # read-back of the set's last results finished
 
-    def one():
-        pb.q_br.copy_(h["q"], non_blocking=True)
-        pb.k_br.copy_(h["k"], non_blocking=True)
-        pb.v_br.copy_(h["v"], non_blocking=True)
-        pb.anchors.copy_(h["anc"], non_blocking=True)
-        pb.z_t[T: T + R].copy_(h["zt_br"], non_blocking=True)
-        for b, row in enumerate(anchor_rows):
-            pb.z_t[row].copy_(h["zt_anc"][b], non_blocking=True)
-        pb.z_d.copy_(h["zd"], non_blocking=True)
+    def one(i):
+        s = i & 1
+        b = sets[s]
+        with torch.cuda.stream(up):
+            if done[s] is not None:
+                up.wait_event(done[s])
+            b["q_br"].copy_(h["q"], non_blocking=True)
+            b["k_br"].copy_(h["k"], non_blocking=True)
+            b["v_br"].copy_(h["v"], non_blocking=True)
+            b["anchors"].copy_(h["anc"], non_blocking=True)
+            b["z_t"][T: T + R].copy_(h["zt_br"], non_blocking=True)
+            for j, row in enumerate(anchor_rows):
+                b["z_t"][row].copy_(h["zt_anc"][j], non_blocking=True)
+            b["z_d"].copy_(h["zd"], non_blocking=True)
+            ready = ev()
+            ready.record(up)
+        comp.wait_event(ready)
+        if copied[s] is not None:
+            comp.wait_event(copied[s])
+        for n in names:
+            setattr(pb, n, b[n])
         pb.step()
-        grad_h.copy_(pb.grad, non_blocking=True)
-        out_h.copy_(pb.out, non_blocking=True)
-        loss_h.copy_(pb.loss, non_blocking=True)
+        d = ev()
+        d.record(comp)
+        done[s] = d
+        with torch.cuda.stream(down):
+            down.wait_event(d)
+            outs[s]["grad"].copy_(b["grad"], non_blocking=True)
+            outs[s]["out"].copy_(b["out"], non_blocking=True)
+            outs[s]["loss"].copy_(b["loss"], non_blocking=True)
+            c = ev()
+            c.record(down)
+        copied[s] = c
 
-    for _ in range(2):
-        one()
+    for i in range(2):
+        one(i)
     torch.cuda.synchronize()
     steps = max(2, min(args.steps, 10))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    e0.record(comp)
+    up.wait_event(e0)
+    for i in range(steps):
+        one(i)
+    comp.wait_event(copied[0])
+    comp.wait_event(copied[1])
+    e1.record(comp)
     torch.cuda.synchronize()
+    for n in names:  # the bench's own buffers again
+        setattr(pb, n, sets[0][n])
     ms = e0.elapsed_time(e1) / steps
     t = torch.tensor([ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
-    ok = bool(torch.isfinite(grad_h).all()) and abs(float(loss_h.item()) - float(pb.loss.item())) == 0
+    last = outs[(steps - 1) & 1]
+    ok = bool(torch.isfinite(last["grad"]).all()) and \
+        abs(float(last["loss"].item()) - float(pb.loss.item())) == 0
     return {"value": pb.R * world / (ms / 1e3), "unit": "rows/s", "ms_per_step": ms,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "pipelined": "two buffer sets; uploads, step and read-back on three streams",
             "results_read_back": ["grad_draft (fp32)", "attention out", "loss"],
             "read_back_finite": ok}
 

@@ -723,20 +723,13 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float mm = -INFINITY;
         for (int cc = 0; cc < nact; ++cc)
           mm = fmaxf(mm, __ldcg(pbase + cc * slot_floats + 128 * D + mrow));
-        // this chunk's own partial first: it is still in TMEM and registers
-        const float wown = (m == -INFINITY) ? 0.f : exp2f(m - mm);
-        float ll = wown * l;
+        // Fixed chunk order 0 .. nact-1 whichever chunk merges: the result
+        // does not depend on the arrival order (bit for bit).
+        float ll = 0.f;
         float acc[D];
 #pragma unroll
-        for (int q = 0; q < DC; ++q) {
-          uint32_t ov[32];
-          tmem_ld32(tO + lane_off + q * 32, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) acc[q * 32 + e] = wown * __uint_as_float(ov[e]);
-        }
+        for (int e = 0; e < D; ++e) acc[e] = 0.f;
         for (int cc = 0; cc < nact; ++cc) {
-          if (cc == c) continue;  // added first, above
           const float* pc = pbase + cc * slot_floats;
           const float mc = __ldcg(pc + 128 * D + mrow);
           const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - mm);
