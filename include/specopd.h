@@ -86,7 +86,10 @@ int specopd_version(void);
 /*
  * Reads the status word of the current device into *host_out and clears it.
  * Synchronises `stream` first.  Returns SPECOPD_OK, or SPECOPD_ERR_CUDA if
- * the copy failed.
+ * the copy failed.  The word is one per device, shared by every call
+ * whatever its stream: with calls in flight on several streams a set bit
+ * says that one of them met the condition (their outputs carry the NaN);
+ * to attribute it to a call, synchronise the other streams first.
  */
 specopd_status specopd_get_device_status(uint32_t* host_out, void* stream);
 
