@@ -676,9 +676,17 @@ cudaError_t launch_row(const TVProblem& p, bool aligned, const void* z_target,
   const tvrow::RowLayout L = row_layout(p);
   if (ws_bytes < L.total) return cudaErrorNotSupported;
   void* fn = pick_row_kernel(p.logit_dtype, p.grad_dtype);
-  const size_t smem = ((sizeof(tvrow::Shared) + 127) / 128) * 128 + (size_t)kStages * 2 * kChunkBytes;
-  int dev = 0, per_sm = 0, nsm = 148;
+  int dev = 0, per_sm = 0, nsm = 148, optin = 0;
   cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  // Pass B's [q < p] bits stay in shared memory after the ring when they
+  // fit (one byte per chunk, vector and consumer thread): pass C then reads
+  // the draft row only.
+  const long long ce_b = (long long)kConsumers * kVPT * (16 / elt_size(p.logit_dtype));
+  const size_t bits_bytes = (size_t)((p.V + ce_b - 1) / ce_b) * kVPT * kConsumers;
+  size_t smem = ((sizeof(tvrow::Shared) + 127) / 128) * 128 + (size_t)kStages * 2 * kChunkBytes;
+  const bool use_bits = p.compute_grad && grad != nullptr && smem + bits_bytes <= (size_t)optin;
+  if (use_bits) smem += (bits_bytes + 15) / 16 * 16;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -699,6 +707,7 @@ cudaError_t launch_row(const TVProblem& p, bool aligned, const void* z_target,
   RowArgs A;
   A.nbranch = p.nbranch; A.W = p.W; A.V = p.V; A.N = p.N; A.rows_target = p.rows_target;
   A.compute_grad = p.compute_grad && grad != nullptr;
+  A.bits = use_bits ? 1 : 0;
   A.norm = p.norm_count;
   A.inv_norm = (float)(1.0 / p.norm_count);
   A.zt = z_target; A.trow = target_row; A.zd = z_draft;

@@ -83,6 +83,7 @@ inline RowLayout row_layout(const TVProblem& p) {
 
 struct RowArgs {
   int nbranch, W, V, N, rows_target, compute_grad;
+  int bits;  // 1: pass B keeps [q < p] per element in shared memory; pass C reads the draft row only
   float inv_norm;
   double norm;
   const void* zt;
@@ -137,6 +138,10 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
   extern __shared__ __align__(128) unsigned char row_smem[];
   Shared& sh = *reinterpret_cast<Shared*>(row_smem);
   uint8_t* ring = row_smem + ((sizeof(Shared) + 127) / 128) * 128;  // [stage][target | draft]
+  // [q < p] of this task's elements, one byte per (chunk, vector, consumer
+  // thread), written by pass B and read by pass C of the same thread (when
+  // A.bits; the buffer follows the ring)
+  uint8_t* bitbuf = ring + (size_t)kStages * 2 * kChunkBytes;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int VN = Vec<Tin>::kN;  // elements per 16-byte vector
   constexpr int VP = Vec<Tin>::kPairs;
@@ -200,6 +205,23 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
         bulk_g2s_hint(dst + kChunkBytes, rd + e0, bytes, &sh.full[st], pol);
         ++q;
       };
+      // pass C with the [q < p] bits: the draft row's chunk only
+      auto issue_d = [&](const Tin* rd, int c, uint64_t pol) {
+        if (!live) return;
+        const int st = (int)(q % kStages);
+        const unsigned use = q / kStages;
+        if (use > 0u && !mbar_wait(&sh.empty[st], (use - 1u) & 1u)) {
+          atomicExch(&A.ctl[2], 1u);
+          live = false;
+          return;
+        }
+        const int e0 = c * CE;
+        const unsigned bytes = (unsigned)(min(CE, V - e0) * (int)sizeof(Tin));
+        uint8_t* dst = ring + (size_t)st * 2 * kChunkBytes;
+        mbar_arrive_expect_tx(&sh.full[st], bytes);
+        bulk_g2s_hint(dst + kChunkBytes, rd + e0, bytes, &sh.full[st], pol);
+        ++q;
+      };
       const Tin *rt_prev = zt, *rd_prev = zd;
       for (int k = 0; k <= ntask && live; ++k) {
         // Another warp's wait ran out (abort): issue nothing more.
@@ -213,7 +235,9 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
           rd = zd + (long long)n * V;
         }
         for (int i = -kLag; i < nch; ++i) {
-          if (hasC && i >= 0) issue(rt_prev, rd_prev, i, drop);
+          if (hasC && i >= 0) {
+            if (A.bits) issue_d(rd_prev, i, drop); else issue(rt_prev, rd_prev, i, drop);
+          }
           if (hasA && i + kLag < nch) issue(rt, rd, i + kLag, load);
         }
         if (hasA)
@@ -350,6 +374,14 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
     }
     return in;
   };
+  // The draft row's vector only (pass C with the [q < p] bits).
+  auto take_d = [&](int c, int v, uint4& ud, auto full) -> bool {
+    const int st = (int)(q % kStages);
+    const int vec = v * kConsumers + tid;
+    const bool in = decltype(full)::value || (c * CE + vec * VN < V);
+    if (in) ud = *reinterpret_cast<const uint4*>(ring + (size_t)st * 2 * kChunkBytes + kChunkBytes + vec * 16);
+    return in;
+  };
   // Release chunk q (one arrive per consumer warp) and advance.
   auto give = [&]() {
     __syncwarp();
@@ -389,16 +421,28 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
 #pragma unroll
         for (int v = 0; v < kVPT; ++v) {
           uint4 ut, ud;
-          if (take(i, v, ut, ud, full)) {
-            float2 ft[VP], fd[VP], o[VP];
-            Vec<Tin>::pairs(ut, ft);
+          if (A.bits ? take_d(i, v, ud, full) : take(i, v, ut, ud, full)) {
+            float2 fd[VP], o[VP];
             Vec<Tin>::pairs(ud, fd);
+            if (A.bits) {
+              const unsigned bm = bitbuf[(i * kVPT + v) * kConsumers + tid];
 #pragma unroll
-            for (int p = 0; p < VP; ++p) {
-              const float2 lt = __ffma2_rn(ft[p], L2E, nLtC);
-              const float2 ld = __ffma2_rn(fd[p], L2E, nLdC);
-              const float2 coef = make_float2(ld.x < lt.x ? c1 : c0, ld.y < lt.y ? c1 : c0);
-              o[p] = __fmul2_rn(ex2_pair(ld), coef);
+              for (int p = 0; p < VP; ++p) {
+                const float2 ld = __ffma2_rn(fd[p], L2E, nLdC);
+                const float2 coef = make_float2((bm >> (2 * p)) & 1u ? c1 : c0,
+                                                (bm >> (2 * p + 1)) & 1u ? c1 : c0);
+                o[p] = __fmul2_rn(ex2_pair(ld), coef);
+              }
+            } else {
+              float2 ft[VP];
+              Vec<Tin>::pairs(ut, ft);
+#pragma unroll
+              for (int p = 0; p < VP; ++p) {
+                const float2 lt = __ffma2_rn(ft[p], L2E, nLtC);
+                const float2 ld = __ffma2_rn(fd[p], L2E, nLdC);
+                const float2 coef = make_float2(ld.x < lt.x ? c1 : c0, ld.y < lt.y ? c1 : c0);
+                o[p] = __fmul2_rn(ex2_pair(ld), coef);
+              }
             }
             Tg* dst = gout + i * CE + (v * kConsumers + tid) * VN;
             if constexpr (sizeof(Tg) == 4) {
@@ -569,13 +613,19 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
           Vec<Tin>::pairs(ut, ft);
           Vec<Tin>::pairs(ud, fd);
 #pragma unroll
+          unsigned bm = 0u;
+#pragma unroll
           for (int p = 0; p < VP; ++p) {
             const float2 lt = __ffma2_rn(ft[p], L2E, nLt);
             const float2 ld = __ffma2_rn(fd[p], L2E, nLd);
             const float2 e = make_float2(ex2_fast(fminf(lt.x, ld.x)), ex2_fast(fminf(lt.y, ld.y)));
+            const bool bx = ld.x < lt.x, by = ld.y < lt.y;
             pa2 = __fadd2_rn(pa2, e);
-            ps2 = __fadd2_rn(ps2, make_float2(ld.x < lt.x ? e.x : 0.f, ld.y < lt.y ? e.y : 0.f));
+            ps2 = __fadd2_rn(ps2, make_float2(bx ? e.x : 0.f, by ? e.y : 0.f));
+            bm |= (bx ? 1u : 0u) << (2 * p);
+            bm |= (by ? 1u : 0u) << (2 * p + 1);
           }
+          if (A.bits) bitbuf[(c * kVPT + v) * kConsumers + tid] = (uint8_t)bm;
         }
       }
       give();
