@@ -612,7 +612,6 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
           float2 ft[VP], fd[VP];
           Vec<Tin>::pairs(ut, ft);
           Vec<Tin>::pairs(ud, fd);
-#pragma unroll
           unsigned bm = 0u;
 #pragma unroll
           for (int p = 0; p < VP; ++p) {
