@@ -12,7 +12,12 @@
 //      (no other CTA is involved);
 //   B: the overlap a_n = sum_v min(p_v, q_v) and s_n = sum_{q<p} q_v;
 //      a_n and s_n are published for the branch;
-//   C: after the branch's W overlaps are in, the gradient row.
+//   C: after the branch's W overlaps are in, the gradient row.  Pass B keeps
+//      [q < p] of every element in shared memory (one byte per chunk,
+//      vector and consumer thread, beside the ring) when it fits, and pass C
+//      then copies the draft row only: five row reads per entry instead of
+//      six, which is what the kernel is bound by (the latency of the
+//      ring's copies, not instruction issue or DRAM bandwidth).
 // The passes of consecutive tasks are pipelined: phase k interleaves pass A
 // of task k with pass C of task k - 1 chunk by chunk (A leads by kLag
 // chunks), then runs pass B of task k.  So each phase reads new rows from
