@@ -254,6 +254,7 @@ def test_tv_8b_bf16_through_score_rows(lib):
     (151_936, 16, 3, "bf16", "f32"),  # the long trunk's vocabulary and W (NS = 12)
     (248_320, 16, 4, "bf16", "f32"),  # the packed batch's vocabulary and W
     (4096, 160, 1, "bf16", "f32"),   # W above the SM count: the slice schedule, aligned rows
+    (140_000, 4, 3, "f32", "f32"),   # fp32 rows too long for pass B's bits: pass C reads both rows
 ])
 def test_tv_shapes(lib, V, W, nb, dtype, gdt):
     rng = np.random.default_rng(V + W)
