@@ -694,8 +694,8 @@ cudaError_t launch_row(const TVProblem& p, bool aligned, const void* z_target,
   if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
   if (e != cudaSuccess) return e;
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  // One CTA per SM keeps the rows in flight within the L2.
-  const long long resident = (long long)std::min(per_sm, 1) * nsm;
+  // Two CTAs per SM (the kernel's geometry).
+  const long long resident = (long long)std::min(per_sm, 2) * nsm;
   if (p.W > resident) return cudaErrorNotSupported;
   const long long G = resident / p.W * p.W;  // whole branches per round
   const int grid = (int)std::min<long long>(G, p.N);
@@ -752,7 +752,7 @@ bool rows_aligned(const TVProblem& p, const void* z_target, const void* z_draft,
          (!cg || (size_t)p.V * gs % 16 == 0);
 }
 
-// Whether the whole-row schedule runs this problem (one CTA per SM, rounds
+// Whether the whole-row schedule runs this problem (two CTAs per SM, rounds
 // of whole branches).
 bool row_applies(const TVProblem& p) {
   void* fn = pick_row_kernel(p.logit_dtype, p.grad_dtype);
@@ -766,7 +766,7 @@ bool row_applies(const TVProblem& p) {
     return false;
   }
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  return p.W <= (long long)std::min(per_sm, 1) * nsm;
+  return p.W <= (long long)std::min(per_sm, 2) * nsm;
 }
 
 }  // namespace

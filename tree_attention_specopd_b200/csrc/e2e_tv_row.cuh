@@ -29,7 +29,7 @@
 //
 // Roles: one producer warp issues the 1-D bulk copies (TMA) of every chunk
 // ahead of the consumers (pass A at normal L2 priority, pass B evict-last,
-// pass C evict-first); 24 consumer warps do the arithmetic; one scorer warp
+// pass C evict-first); 12 consumer warps do the arithmetic; one scorer warp
 // publishes each task's (a_n, s_n) from the consumer warps' partials, waits
 // for the branch, computes g_n and the owner's outputs, and hands g_n to the
 // consumers through an mbarrier.
@@ -38,19 +38,21 @@
 // W and at most the resident CTAs, so every round holds whole branches.  A
 // task's handshake waits only for the other positions of its branch, which
 // run on resident CTAs of the same round and publish after pass B, which
-// needs only earlier handshakes of the same CTAs: no deadlock.  One CTA per
-// SM keeps the rows in flight within the L2.  Every wait is bounded.
+// needs only earlier handshakes of the same CTAs: no deadlock.  Two CTAs
+// share an SM (12 consumer warps, a 72 KB ring and the pass-B bits each):
+// two positions in flight per SM, each ring coupling fewer warps (measured
+// 3 % faster at 8B than one CTA of 24 warps with a 192 KB ring).  Every wait
+// is bounded.
 
 namespace tvrow {
 
-constexpr int kConsumers = 768;              // 24 consumer warps
+constexpr int kConsumers = 384;              // 12 consumer warps (two CTAs per SM)
 constexpr int kCWarps = kConsumers / 32;
 constexpr int kProducerWarp = kCWarps;       // issues the bulk copies
 constexpr int kScorerWarp = kCWarps + 1;     // branch handshake, g_n, owner outputs, loss
 constexpr int kThreads = kConsumers + 64;
 constexpr int kVPT = 1;                      // 16-byte vectors per consumer per row per chunk
-constexpr int kStages = 8;                   // ring depth (8 x 24 KB; finer stages measured
-                                             // 2-4 % faster than 4 x 48 KB)
+constexpr int kStages = 6;                   // ring depth (6 x 12 KB)
 constexpr int kChunkBytes = kConsumers * 16 * kVPT;  // bytes of one row per chunk
 constexpr int kMaxW = 256;
 constexpr int kLag = 4;                      // pass-A chunks ahead of pass C in a phase
@@ -138,7 +140,7 @@ __device__ __forceinline__ void warp_lse2_merge(float& m, float& s) {
 }  // namespace tvrow
 
 template <typename Tin, typename Tg>
-__global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tvrow::RowArgs A) {
+__global__ void __launch_bounds__(tvrow::kThreads, 2) e2e_tv_row_kernel(const tvrow::RowArgs A) {
   using namespace tvrow;
   extern __shared__ __align__(128) unsigned char row_smem[];
   Shared& sh = *reinterpret_cast<Shared*>(row_smem);
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
       int last = 0;
       int ok_branch = 0;
       if (lane == 0) {
-        // publish (a_n, s_n) once the 24 consumer warps' partials are in
+        // publish (a_n, s_n) once every consumer warp's partials are in
         const bool in = mbar_wait(&sh.bdone, (unsigned)(k & 1));
         float2 v = make_float2(qnan, qnan);
         if (in) {
@@ -575,7 +577,7 @@ __global__ void __launch_bounds__(tvrow::kThreads, 1) e2e_tv_row_kernel(const tv
     if (!hasA) break;  // the last phase held only the last gradient row
 
     // ------------------------------ lse of task k
-    // Every warp waits for the 24 records (bounded), then combines them
+    // Every warp waits for the kCWarps records (bounded), then combines them
     // itself.  The combination is symmetric in its two operands, so the
     // butterfly leaves the same bits in every lane, and every warp computes
     // the same L.  The records alternate between two buffers by task parity:
