@@ -255,6 +255,7 @@ def test_tv_8b_bf16_through_score_rows(lib):
     (248_320, 16, 4, "bf16", "f32"),  # the packed batch's vocabulary and W
     (4096, 160, 1, "bf16", "f32"),   # W above the SM count: the slice schedule, aligned rows
     (140_000, 4, 3, "f32", "f32"),   # fp32 rows too long for pass B's bits: pass C reads both rows
+    (50_000, 4, 5, "bf16", "bf16"),  # whole-row schedule, pass-C bits, bf16 gradient rows
 ])
 def test_tv_shapes(lib, V, W, nb, dtype, gdt):
     rng = np.random.default_rng(V + W)
