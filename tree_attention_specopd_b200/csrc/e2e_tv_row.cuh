@@ -55,7 +55,7 @@ constexpr int kVPT = 1;                      // 16-byte vectors per consumer per
 constexpr int kStages = 6;                   // ring depth (6 x 12 KB)
 constexpr int kChunkBytes = kConsumers * 16 * kVPT;  // bytes of one row per chunk
 constexpr int kMaxW = 256;
-constexpr int kLag = 4;                      // pass-A chunks ahead of pass C in a phase
+constexpr int kLag = 8;                      // pass-A chunks ahead of pass C in a phase
 
 struct Shared {
   uint64_t full[kStages], empty[kStages];
