@@ -261,61 +261,6 @@ __device__ __forceinline__ void rope_row_smem(uint8_t* lo_line, uint8_t* hi_line
   }
 }
 
-// The same rotation for a query line of a tile whose G query heads share a
-// branch row (G a power of two up to 8, so the G lines of a row are G
-// consecutive lanes of one warp, all at the same position): lane g of a
-// group forms the angles of frequencies t = g, g + G, ... of each 8-pair
-// chunk and the group exchanges them by shuffle, so each angle is reduced
-// and evaluated once per row instead of G times.  Called by all 32 lanes;
-// `active` lanes rotate their line.  Bit-identical to rope_row_smem.
-template <int D, int G>
-__device__ __forceinline__ void rope_row_smem_group(uint8_t* lo_line, uint8_t* hi_line, int line,
-                                                    int pos, const double* theta, bool active) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_two_pi = 0.15915494309189533576888376337251;
-  const int lane = threadIdx.x & 31;
-  const int g = lane & (G - 1), base = lane & ~(G - 1);
-  const int sw = line & 7;
-  for (int c = 0; c < D / 16; ++c) {
-    float cm[8 / G], sm[8 / G];
-#pragma unroll
-    for (int j = 0; j < 8 / G; ++j) {
-      const double ang = (double)pos * theta[8 * c + g + j * G];
-      const float red = (float)(ang - two_pi * rint(ang * inv_two_pi));
-      __sincosf(red, &sm[j], &cm[j]);
-    }
-    float cs[8], sn[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      cs[t] = __shfl_sync(0xffffffffu, cm[t / G], base + (t % G));
-      sn[t] = __shfl_sync(0xffffffffu, sm[t / G], base + (t % G));
-    }
-    if (active) {
-      uint4* pa = reinterpret_cast<uint4*>(lo_line + ((c ^ sw) << 4));
-      uint4* pb = reinterpret_cast<uint4*>(hi_line + (((D == 128 ? c : c + 4) ^ sw) << 4));
-      const uint4 a = *pa, b = *pb;
-      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
-      uint32_t ra[4], rb[4];
-#pragma unroll
-      for (int e2 = 0; e2 < 4; ++e2) {
-        float ya[2], yb[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float c_ = cs[2 * e2 + h], s_ = sn[2 * e2 + h];
-          const float xa = h ? bf16hi(wa[e2]) : bf16lo(wa[e2]);
-          const float xb = h ? bf16hi(wb[e2]) : bf16lo(wb[e2]);
-          ya[h] = xa * c_ - xb * s_;
-          yb[h] = xb * c_ + xa * s_;
-        }
-        ra[e2] = pack_bf16x2(ya[0], ya[1]);
-        rb[e2] = pack_bf16x2(yb[0], yb[1]);
-      }
-      *pa = make_uint4(ra[0], ra[1], ra[2], ra[3]);
-      *pb = make_uint4(rb[0], rb[1], rb[2], rb[3]);
-    }
-  }
-}
-
 // ------------------------------------------------------------------ kernel
 template <int D>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
@@ -590,18 +535,9 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // Q line), then half a line of each leading branch key tile.  The
       // async proxy (tcgen05.mma) reads them after the fence and rot_done.
       bool okr = warp_wait_or_abort(&hdr->q_full, 0, hdr);
-      uint8_t* qlo = sQ + mrow * 128;
-      uint8_t* qhi = sQ + (D == 128 ? kQHalf : 0) + mrow * 128;
-      if (okr) {  // warp-uniform: the grouped forms shuffle across the warp
-        if (G == 4)
-          rope_row_smem_group<D, 4>(qlo, qhi, mrow, qpos, P.theta, in_tile);
-        else if (G == 8)
-          rope_row_smem_group<D, 8>(qlo, qhi, mrow, qpos, P.theta, in_tile);
-        else if (G == 2)
-          rope_row_smem_group<D, 2>(qlo, qhi, mrow, qpos, P.theta, in_tile);
-        else if (in_tile)
-          rope_row_smem<D>(qlo, qhi, mrow, qpos, P.theta, 0, D / 16);
-      }
+      if (okr && in_tile)
+        rope_row_smem<D>(sQ + mrow * 128, sQ + (D == 128 ? kQHalf : 0) + mrow * 128, mrow, qpos,
+                         P.theta, 0, D / 16);
       const int t128 = tid - 64;  // 0..127
       for (int j = 0; j < nbt; ++j) {
         // branch tile j sits in K stage j (nbt <= 2 < kKStages), first use
