@@ -22,6 +22,10 @@ What it computes, and from which passage (pages on arXiv 2611.02846):
 * ``oracle.tv``         -- E2E-TV: overlap a = sum min(p, q) = 1 - TV,
   prefix products, loss 1 - mean prefix product, closed-form gradient with
   respect to the draft logits.  Review §1.1 and §3.3; summary §2.3.
+* ``oracle.lmhead``     -- the same E2E-TV with the logits formed from hidden
+  rows through the target's and the drafter's LM heads (z = W h), target
+  rows gathered by the score-row map.  Review §3.2(a) (score-row reading
+  rule) and §3.3.
 
 Parity pins (tests/test_oracle_*.py, run with ``-m "not gpu"``) tie every
 function to facts the pages or mathematics fix; see those tests.  Parity
@@ -29,6 +33,6 @@ unpinned: none of the functions here (the only unpinned figure of the pages,
 the 69.2x attention-pair ratio, is not computed by the oracle).
 """
 
-from . import attention, tree, tv  # noqa: F401
+from . import attention, lmhead, tree, tv  # noqa: F401
 
-__all__ = ["attention", "tree", "tv"]
+__all__ = ["attention", "lmhead", "tree", "tv"]
