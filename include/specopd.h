@@ -12,6 +12,8 @@
  *                       cached trunk K/V and their own branch history
  *   specopd_e2e_tv      per-position overlap a = sum_v min(p_v, q_v), branch
  *                       prefix products, loss and d loss / d draft logits
+ *   specopd_e2e_tv_lmhead  the same from hidden rows and the two LM heads,
+ *                       the logits formed on chip and never stored
  *
  * Sources (web pages on arXiv 2611.02846, cited by title and section):
  *   [review]  "SpecOPD: Branch-Parallel On-Policy Distillation for
@@ -314,6 +316,56 @@ specopd_status specopd_e2e_tv(const specopd_tv_desc* desc,
  */
 specopd_status specopd_e2e_tv_finalize(const double* numer_sum, int64_t norm_count,
                                        float* loss, double* loss64, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* E2E-TV with the LM heads fused in front: [review §3.2(a)] (score-row
+ * reading rule: the logits that score position n come from the output of
+ * its predictor row, target_row[n]) and [review §3.3] (E2E-TV on those
+ * logits).  The logits are formed tile by tile on the tensor cores from the
+ * hidden rows and the two heads and never stored:
+ *   z_t[n] = W_target h_target[target_row[n]],   z_d[n] = W_draft h_draft[n]
+ * (fp32 accumulation of bf16 products; no bias, norm or temperature), then
+ * a, prefix, numer, loss and grad_draft = d loss / d z_d exactly as
+ * specopd_e2e_tv defines them.  Three passes over the heads (statistics,
+ * overlaps, gradient), each reading both heads once.
+ */
+typedef struct {
+  int nbranch;               /* S*B branches                                 */
+  int W;                     /* positions per branch, 1 .. 256               */
+  int V;                     /* vocabulary size (rows of each head)          */
+  int d_model;               /* hidden size, a multiple of 8                 */
+  int rows_target;           /* rows of h_target (bounds for target_row)     */
+  specopd_dtype grad_dtype;  /* grad_draft                                   */
+  int compute_grad;          /* 0: skip grad_draft (two passes instead of 3) */
+  int64_t norm_count;        /* divisor of the loss; 0 -> nbranch*W          */
+} specopd_lmhead_tv_desc;
+
+/* Bytes of workspace specopd_e2e_tv_lmhead needs (>= 256; depends on the
+ * current device's SM count). */
+size_t specopd_e2e_tv_lmhead_workspace_size(const specopd_lmhead_tv_desc* desc);
+
+/*
+ * h_target    bf16 [rows_target, d_model] target hidden rows
+ * target_row  device int32[N] row of h_target scoring position n, or NULL for
+ *             the identity (rows_target must then be >= N)
+ * w_target    bf16 [V, d_model] target LM head (row v scores token v)
+ * h_draft     bf16 [N, d_model] draft hidden rows, branch-major (b, i)
+ * w_draft     bf16 [V, d_model] draft LM head
+ * a, prefix   device fp32[N]; loss device fp32[1]; numer fp64[1] or NULL
+ * grad_draft  [N, V] (grad_dtype) or NULL; required when compute_grad != 0;
+ *             16-byte aligned with V * element size a multiple of 16
+ * The four bf16 matrices must start on 16-byte boundaries.  A target_row
+ * outside [0, rows_target) sets SPECOPD_DEV_ROW_RANGE and makes NaN that
+ * position's a, its branch's prefix products from it on, its branch's
+ * gradient rows and the loss; a bounded wait that runs out sets
+ * SPECOPD_DEV_TIMEOUT.
+ */
+specopd_status specopd_e2e_tv_lmhead(const specopd_lmhead_tv_desc* desc,
+                                     const void* h_target, const int32_t* target_row,
+                                     const void* w_target, const void* h_draft,
+                                     const void* w_draft, float* a, float* prefix,
+                                     float* loss, double* numer, void* grad_draft,
+                                     void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* E2E-TV for callers that cannot allocate device memory.  The paper has no

@@ -17,6 +17,11 @@ Recipe (NumPy PCG64, seed 0 unless stated):
     distinct uniform ids ("peaked tokens"); draft row = target row +
     N(0, sigma_d).  The overlap sweep adds 5% bit-identical rows and 5% rows
     whose draft and target have disjoint top-20 supports.
+  * LM-head inputs (hidden rows and heads): target head W_t ~ N(0, (sigma /
+    sqrt(d))^2), draft head W_d = W_t + N(0, (rho sigma / sqrt(d))^2); target
+    hidden rows ~ N(0, 1); the draft row of position n = the target row it is
+    scored against + N(0, rho^2).  So logits have spread about sigma and the
+    two models agree partly.  All rounded to bf16.
 """
 
 from __future__ import annotations
@@ -246,3 +251,30 @@ def logits(cfg: TVConfig, positions=None):
     for i, n in enumerate(positions):
         zt[i], zd[i] = logit_rows(cfg, n)
     return zt, zd
+
+
+# --------------------------------------------------------------------------
+# LM-head inputs
+
+@dataclass
+class LmheadInputs:
+    h_target: np.ndarray    # f32 [rows_target, d], bf16-exact
+    target_row: np.ndarray  # int32 [N]
+    w_target: np.ndarray    # f32 [V, d], bf16-exact
+    h_draft: np.ndarray     # f32 [N, d], bf16-exact
+    w_draft: np.ndarray     # f32 [V, d], bf16-exact
+
+
+def lmhead_inputs(seed, nbranch, W, V, d, rows_target=None, sigma=3.0, rho=0.5):
+    """Seeded hidden rows and LM heads (see the module recipe).  target_row is
+    a random injective map of the N positions into [0, rows_target)."""
+    N = nbranch * W
+    rows_target = N if rows_target is None else rows_target
+    rng = np.random.default_rng(seed)
+    sc = sigma / np.sqrt(d)
+    w_t = rng.standard_normal((V, d), dtype=np.float32) * np.float32(sc)
+    w_d = w_t + rng.standard_normal((V, d), dtype=np.float32) * np.float32(rho * sc)
+    h_t = rng.standard_normal((rows_target, d), dtype=np.float32)
+    trow = rng.permutation(rows_target)[:N].astype(np.int32)
+    h_d = h_t[trow] + rng.standard_normal((N, d), dtype=np.float32) * np.float32(rho)
+    return LmheadInputs(round_bf16(h_t), trow, round_bf16(w_t), round_bf16(h_d), round_bf16(w_d))

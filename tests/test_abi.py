@@ -20,7 +20,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = api.header_functions()
-    assert len(names) == 14
+    assert len(names) == 16
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
@@ -70,3 +70,26 @@ def test_bf16_branch_span_limit(lib):
     args = [fake] * 5 + [fake, cu, fake, fake, fake, None, fake, 1 << 20, None]
     d = api.attn_desc(1, 4, 70, 8, 8, 128, "bf16")  # G = 1: 128 + 68 = 196 > 192
     assert lib.specopd_tree_attn(ctypes.byref(d), *args) == 2  # SPECOPD_ERR_UNSUPPORTED
+
+
+def test_lmhead_tv_validation(lib):
+    # specopd_e2e_tv_lmhead: descriptor and pointer checks come before any
+    # device work.
+    ok = api.lmhead_tv_desc(64, 8, 151936, 4096, 512)
+    assert api.specopd_e2e_tv_lmhead_workspace_size(ok) >= 512 * 4096 * 2
+    assert api.specopd_e2e_tv_lmhead_workspace_size(api.lmhead_tv_desc(0, 8, 100, 64, 8)) == 0
+    fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    ptrs = [fake, None, fake, fake, fake, fake, fake, fake, None, fake, fake, 1 << 30, None]
+    bad_d = api.lmhead_tv_desc(2, 4, 1000, 100, 8)  # hidden size not a multiple of 8
+    assert lib.specopd_e2e_tv_lmhead(ctypes.byref(bad_d), *ptrs) == 2  # UNSUPPORTED
+    bad_w = api.lmhead_tv_desc(2, 300, 1000, 64, 600)  # W above 256
+    assert lib.specopd_e2e_tv_lmhead(ctypes.byref(bad_w), *ptrs) == 2
+    d = api.lmhead_tv_desc(2, 4, 1000, 64, 8)
+    missing = list(ptrs)
+    missing[2] = None  # no target head
+    assert lib.specopd_e2e_tv_lmhead(ctypes.byref(d), *missing) == 1  # INVALID_ARG
+    unaligned = list(ptrs)
+    unaligned[0] = ctypes.c_void_p(264)  # h_target off a 16-byte boundary
+    assert lib.specopd_e2e_tv_lmhead(ctypes.byref(d), *unaligned) == 2
+    rows = api.lmhead_tv_desc(2, 4, 1000, 64, 7)  # identity rows need rows_target >= N
+    assert lib.specopd_e2e_tv_lmhead(ctypes.byref(rows), *ptrs) == 1

@@ -8,6 +8,8 @@ from . import api  # noqa: F401
 from .api import (  # noqa: F401
     SpecopdError,
     specopd_e2e_tv,
+    specopd_e2e_tv_lmhead,
+    specopd_e2e_tv_lmhead_workspace_size,
     specopd_e2e_tv_workspace_size,
     specopd_get_device_status,
     specopd_rope_apply,

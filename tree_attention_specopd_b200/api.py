@@ -52,6 +52,13 @@ class TVDesc(ctypes.Structure):
                 ("norm_count", ctypes.c_int64)]
 
 
+class LmheadTVDesc(ctypes.Structure):
+    _fields_ = [("nbranch", ctypes.c_int), ("W", ctypes.c_int), ("V", ctypes.c_int),
+                ("d_model", ctypes.c_int), ("rows_target", ctypes.c_int),
+                ("grad_dtype", ctypes.c_int), ("compute_grad", ctypes.c_int),
+                ("norm_count", ctypes.c_int64)]
+
+
 _lib = None
 
 
@@ -97,6 +104,11 @@ def load(path: str = LIB_PATH):
     lib.specopd_e2e_tv_noalloc.restype = cint
     lib.specopd_e2e_tv_noalloc.argtypes = [ctypes.POINTER(TVDesc), vp, i32p, vp, f32p, f32p,
                                            f32p, f64p, vp, vp]
+    lib.specopd_e2e_tv_lmhead_workspace_size.restype = csize
+    lib.specopd_e2e_tv_lmhead_workspace_size.argtypes = [ctypes.POINTER(LmheadTVDesc)]
+    lib.specopd_e2e_tv_lmhead.restype = cint
+    lib.specopd_e2e_tv_lmhead.argtypes = [ctypes.POINTER(LmheadTVDesc), vp, i32p, vp, vp, vp,
+                                          f32p, f32p, f32p, f64p, vp, vp, csize, vp]
     lib.specopd_e2e_tv_finalize.restype = cint
     lib.specopd_e2e_tv_finalize.argtypes = [f64p, ctypes.c_int64, f32p, f64p, vp]
     lib.specopd_debug_fault_injection.restype = cint
@@ -255,6 +267,47 @@ def specopd_e2e_tv(desc, z_target, target_row, z_draft, a=None, prefix=None, los
                                  _ptr(z_draft), _ptr(a), _ptr(prefix), _ptr(loss), _ptr(numer),
                                  _ptr(grad), _ptr(workspace), workspace.numel(), _stream(stream)),
            "e2e_tv")
+    return {"a": a, "prefix": prefix, "loss": loss, "numer": numer, "grad": grad}
+
+
+def lmhead_tv_desc(nbranch, W, V, d_model, rows_target, grad_dtype="f32", compute_grad=True,
+                   norm_count=0):
+    g = grad_dtype if isinstance(grad_dtype, int) else (
+        BF16 if grad_dtype in ("bf16", torch.bfloat16) else F32)
+    return LmheadTVDesc(nbranch, W, V, d_model, rows_target, g, 1 if compute_grad else 0,
+                        int(norm_count))
+
+
+def specopd_e2e_tv_lmhead_workspace_size(desc) -> int:
+    return int(load().specopd_e2e_tv_lmhead_workspace_size(ctypes.byref(desc)))
+
+
+def specopd_e2e_tv_lmhead(desc, h_target, target_row, w_target, h_draft, w_draft, a=None,
+                          prefix=None, loss=None, numer=None, grad=None, workspace=None,
+                          stream=None):
+    """E2E-TV from bf16 hidden rows and LM heads.  Returns dict(a, prefix,
+    loss, numer, grad)."""
+    dev = h_draft.device
+    N = desc.nbranch * desc.W
+    if a is None:
+        a = torch.empty(N, dtype=torch.float32, device=dev)
+    if prefix is None:
+        prefix = torch.empty(N, dtype=torch.float32, device=dev)
+    if loss is None:
+        loss = torch.empty(1, dtype=torch.float32, device=dev)
+    if numer is None:
+        numer = torch.empty(1, dtype=torch.float64, device=dev)
+    if grad is None and desc.compute_grad:
+        gdt = torch.bfloat16 if desc.grad_dtype == BF16 else torch.float32
+        grad = torch.empty((N, desc.V), dtype=gdt, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(specopd_e2e_tv_lmhead_workspace_size(desc), 256),
+                                dtype=torch.uint8, device=dev)
+    _check(load().specopd_e2e_tv_lmhead(ctypes.byref(desc), _ptr(h_target), _ptr(target_row),
+                                        _ptr(w_target), _ptr(h_draft), _ptr(w_draft), _ptr(a),
+                                        _ptr(prefix), _ptr(loss), _ptr(numer), _ptr(grad),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+           "e2e_tv_lmhead")
     return {"a": a, "prefix": prefix, "loss": loss, "numer": numer, "grad": grad}
 
 

@@ -15,6 +15,7 @@
 #include "rope.cu"
 #include "tree_attn_simt.cu"
 #include "tree_attn_sm100.cu"
+#include "lmhead_tv.cu"
 #include "tree_build.cu"
 
 using namespace specopd;
@@ -156,6 +157,24 @@ specopd_status e2e_tv_checked(const specopd_tv_desc* d, const void* z_target,
                                 workspace, ws_bytes, as_stream(stream));
   if (e == cudaErrorInvalidConfiguration) { cudaGetLastError(); return SPECOPD_ERR_UNSUPPORTED; }
   return cuda_status(e);
+}
+
+specopd_status lmtv_problem(const specopd_lmhead_tv_desc* d, LmtvProblem& p) {
+  if (!d) return SPECOPD_ERR_INVALID_ARG;
+  if (d->nbranch < 1 || d->W < 1 || d->V < 1 || d->d_model < 1 || d->rows_target < 1)
+    return SPECOPD_ERR_INVALID_ARG;
+  if (d->grad_dtype != SPECOPD_F32 && d->grad_dtype != SPECOPD_BF16) return SPECOPD_ERR_INVALID_ARG;
+  if (d->norm_count < 0) return SPECOPD_ERR_INVALID_ARG;
+  // rows of the hidden states and heads must be whole 16-byte units (TMA)
+  if (d->d_model % 8 != 0 || d->W > 256) return SPECOPD_ERR_UNSUPPORTED;
+  const long long N = (long long)d->nbranch * d->W;
+  if (N > (1ll << 30)) return SPECOPD_ERR_UNSUPPORTED;
+  p.nbranch = d->nbranch; p.W = d->W; p.V = d->V; p.N = (int)N; p.d = d->d_model;
+  p.rows_target = d->rows_target;
+  p.grad_dtype = d->grad_dtype;
+  p.compute_grad = d->compute_grad ? 1 : 0;
+  p.norm_count = d->norm_count > 0 ? (double)d->norm_count : (double)N;
+  return SPECOPD_OK;
 }
 
 }  // namespace
@@ -365,6 +384,40 @@ specopd_status specopd_debug_fault_injection(int64_t withhold_position,
   if (s != SPECOPD_OK) return s;
   const FaultInject f = {(long long)withhold_position, (unsigned long long)branch_wait_limit_ns};
   return cuda_status(cudaMemcpyToSymbol(specopd::g_inject, &f, sizeof(f)));
+}
+
+size_t specopd_e2e_tv_lmhead_workspace_size(const specopd_lmhead_tv_desc* d) {
+  LmtvProblem p;
+  if (lmtv_problem(d, p) != SPECOPD_OK) return 0;
+  const size_t w = lmtv_workspace(p);
+  return w < 256 ? 256 : w;
+}
+
+specopd_status specopd_e2e_tv_lmhead(const specopd_lmhead_tv_desc* d, const void* h_target,
+                                     const int32_t* target_row, const void* w_target,
+                                     const void* h_draft, const void* w_draft, float* a,
+                                     float* prefix, float* loss, double* numer, void* grad_draft,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  LmtvProblem p;
+  specopd_status s = lmtv_problem(d, p);
+  if (s != SPECOPD_OK) return s;
+  if (!h_target || !w_target || !h_draft || !w_draft || !a || !prefix || !loss)
+    return SPECOPD_ERR_INVALID_ARG;
+  if (p.compute_grad && !grad_draft) return SPECOPD_ERR_INVALID_ARG;
+  if (!target_row && p.rows_target < p.N) return SPECOPD_ERR_INVALID_ARG;
+  if (!aligned16(h_target) || !aligned16(w_target) || !aligned16(h_draft) || !aligned16(w_draft))
+    return SPECOPD_ERR_UNSUPPORTED;
+  const size_t gs = p.grad_dtype == SPECOPD_BF16 ? 2 : 4;
+  if (p.compute_grad && (!aligned16(grad_draft) || ((size_t)p.V * gs) % 16 != 0))
+    return SPECOPD_ERR_UNSUPPORTED;
+  if (!workspace) return SPECOPD_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SPECOPD_ERR_UNSUPPORTED;
+  s = check_device();
+  if (s != SPECOPD_OK) return s;
+  if (ws_bytes < lmtv_workspace(p)) return SPECOPD_ERR_WORKSPACE;
+  return cuda_status(launch_lmtv(p, h_target, target_row, w_target, h_draft, w_draft, a, prefix,
+                                 loss, numer, p.compute_grad ? grad_draft : nullptr, workspace,
+                                 ws_bytes, as_stream(stream)));
 }
 
 }  // extern "C"

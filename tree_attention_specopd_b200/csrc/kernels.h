@@ -86,4 +86,18 @@ cudaError_t launch_e2e_tv(const TVProblem& p, const void* z_target, const int32_
                           const void* z_draft, float* a, float* prefix, float* loss, double* numer,
                           void* grad, void* ws, size_t ws_bytes, cudaStream_t st);
 
+// E2E-TV with the LM heads fused in front (lmhead_tv.cu): hidden rows and
+// heads in bf16, N = nbranch * W positions, d = hidden size.
+struct LmtvProblem {
+  int nbranch, W, V, N, d, rows_target;
+  specopd_dtype grad_dtype;
+  int compute_grad;
+  double norm_count;
+};
+size_t lmtv_workspace(const LmtvProblem& p);
+cudaError_t launch_lmtv(const LmtvProblem& p, const void* h_target, const int32_t* target_row,
+                        const void* w_target, const void* h_draft, const void* w_draft, float* a,
+                        float* prefix, float* loss, double* numer, void* grad, void* ws,
+                        size_t ws_bytes, cudaStream_t st);
+
 }  // namespace specopd
