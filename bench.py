@@ -330,6 +330,7 @@ def run_gpu(args):
 
     # ---- the other workloads, device-timed in the same run (one GPU)
     extra = None
+    lmhead = None
     if world == 1 and wl == WORKLOAD and not args.no_extra_workloads:
         figs = _Figures(pb)
         del pb
@@ -339,6 +340,7 @@ def run_gpu(args):
             extra[other] = measure_workload(torch, api, dev, other, max(3, min(args.steps, 10)),
                                             args.warmup)
             torch.cuda.empty_cache()
+        lmhead = measure_lmhead_tv(torch, api, dev)
         pb = figs
 
     if rank == 0:
@@ -402,6 +404,8 @@ def run_gpu(args):
         }
         if extra is not None:
             line["workloads"] = extra
+        if lmhead is not None:
+            line["lmhead_tv"] = lmhead
         if e2e is None:
             line["e2e_note"] = "host-buffer end-to-end measured on the default 8B workload only"
         if not args.no_cpu_baseline:
@@ -463,6 +467,55 @@ def measure_workload(torch, api, dev, workload, steps, warmup):
            "l2": "inputs larger than L2" if pb.tv_bytes / 2 > 126e6 else "inputs fit in L2"}
     del pb
     return out
+
+
+def measure_lmhead_tv(torch, api, dev, nbranch=64, W=8, V=151936, d=4096, reps=5, warmup=2):
+    """Device time of specopd_e2e_tv_lmhead (the LM heads fused in front of
+    E2E-TV) on the 8B shape with a 4096-wide hidden state: seeded bf16 hidden
+    rows and heads made on the device with the synth recipe's distributions,
+    CUDA events around `reps` calls after `warmup`.  Executed tensor work:
+    passes 0 and 1 form both models' logits, pass 2 the draft's (5 GEMMs of
+    2 N V d FLOPs)."""
+    N = nbranch * W
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    sc = 3.0 / d ** 0.5
+    wt = (torch.randn(V, d, device=dev, generator=g) * sc).to(torch.bfloat16)
+    wd = (wt.float() + torch.randn(V, d, device=dev, generator=g) * (0.5 * sc)).to(torch.bfloat16)
+    ht = torch.randn(N, d, device=dev, generator=g).to(torch.bfloat16)
+    hd = (ht.float() + 0.5 * torch.randn(N, d, device=dev, generator=g)).to(torch.bfloat16)
+    desc = api.lmhead_tv_desc(nbranch, W, V, d, N, "f32", True)
+    ws = torch.empty(api.specopd_e2e_tv_lmhead_workspace_size(desc), dtype=torch.uint8, device=dev)
+    out = {"a": torch.empty(N, device=dev), "prefix": torch.empty(N, device=dev),
+           "loss": torch.empty(1, device=dev),
+           "numer": torch.empty(1, dtype=torch.float64, device=dev),
+           "grad": torch.empty((N, V), device=dev)}
+    for _ in range(warmup):
+        api.specopd_e2e_tv_lmhead(desc, ht, None, wt, hd, wd, workspace=ws, **out)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        api.specopd_e2e_tv_lmhead(desc, ht, None, wt, hd, wd, workspace=ws, **out)
+    e1.record()
+    torch.cuda.synchronize()
+    st = api.specopd_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x} after specopd_e2e_tv_lmhead")
+    ms = e0.elapsed_time(e1) / reps
+    flops = 5 * 2.0 * N * V * d
+    peaks = _peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    res = {"call": "specopd_e2e_tv_lmhead", "nbranch": nbranch, "W": W, "V": V, "d_model": d,
+           "grad_dtype": "f32", "launch_ms": ms, "executed_flops_per_call": flops,
+           "achieved": tf, "unit": "TFLOP/s", "bound": "tensor", "peak": peaks["bf16_tflops"],
+           "frac": tf / peaks["bf16_tflops"], "peak_src": peaks["src"],
+           "positions_per_s": N / (ms / 1e3),
+           "logit_bytes_not_stored": 2 * N * V * 2}
+    del wt, wd, ht, hd, ws, out
+    torch.cuda.empty_cache()
+    return res
 
 
 TV_SOURCES = (

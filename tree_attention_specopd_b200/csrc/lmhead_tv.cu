@@ -14,21 +14,22 @@
 // B200 design.  Three passes of one tcgen05 GEMM kernel over tiles of 128
 // positions x 128 vocabulary entries, each tile holding both models'
 // logits in TMEM (fp32, 2 x 128 columns, double-buffered: 512 columns, one
-// CTA per SM), with a per-pass epilogue:
+// CTA per SM; pass 2 the draft's only), with a per-pass epilogue:
 //   pass 0: per row, running (max, sum of 2^(x - max)) of both rows over the
 //           CTA's vocabulary chunk -> one record per (chunk, row);
 //   (combine: the chunks' records in chunk order -> lse of both rows)
 //   pass 1: per row, sum_v 2^min(lt, ld) and the [ld < lt] part of it over
 //           the chunk -> one (a, s) record per (chunk, row);
 //   (branch: a_n, s_n in chunk order, prefix products, g_n, the loss)
-//   pass 2: dz_d[n, v] = g_n q_v ([q_v < p_v] - s_n), written as the tile's
-//           epilogue.
-// Passes 1 and 2 recompute the same tiles with the same instructions, so the
-// [q < p] decisions of s_n and of the gradient agree bit for bit.
+//   pass 1 also stores [q_v < p_v] of every entry (one bit; N V / 8 bytes);
+//   pass 2: the draft tiles only, dz_d[n, v] = g_n q_v ([q_v < p_v] - s_n)
+//           with pass 1's bits, written as the tile's epilogue (so s_n and the
+//           gradient's mask are the same decisions).
 //  * Warp 0 drives TMA: per stage a 64-column slice (one 128-byte swizzled
 //    row) of the 128 target rows, of 128 rows of the target head, of the
-//    128 draft rows and of the draft head (4 x 16 KB, 3 stages).  Rows past
-//    N or V and columns past d arrive as zeros.
+//    128 draft rows and of the draft head (4 x 16 KB, 3 stages; pass 2: the
+//    draft's two, 6 stages).  Rows past N or V and columns past d arrive as
+//    zeros.
 //  * Warp 1 issues tcgen05.mma (M = N = 128, K = 16, both operands K-major
 //    from shared memory) from one thread, commits each stage back to the
 //    producer and each finished tile to the epilogue.
@@ -58,15 +59,15 @@ constexpr int kThreads = 192;           // warp 0: TMA, warp 1: MMA + TMEM, warp
 constexpr int kBM = 128;                // positions per tile (TMEM lanes)
 constexpr int kBN = 128;                // vocabulary entries per tile (MMA N)
 constexpr int kBK = 64;                 // hidden columns per stage (one 128-byte swizzled row)
-constexpr int kStages = 3;
 constexpr int kTile = kBM * kBK * 2;    // 16 KB: one operand slice of one stage
-constexpr int kStageBytes = 4 * kTile;  // target rows, target head, draft rows, draft head
+constexpr int kRing = 12 * kTile;       // 192 KB of stages: 3 of both models, 6 of the draft only
+constexpr int kMaxStages = 6;
 constexpr int kTmemCols = 512;          // buffer b: target [256b, 256b+128), draft [256b+128, 256b+256)
 constexpr int kMaxW = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Hdr {
-  uint64_t full[kStages], empty[kStages];
+  uint64_t full[kMaxStages], empty[kMaxStages];
   uint64_t acc_full[2];  // by tile parity: both logit tiles are in TMEM
   uint64_t acc_free[2];  // by tile parity: the epilogue warps have read them
   uint64_t mma_done;     // one phase: every MMA the CTA issued has completed
@@ -80,6 +81,7 @@ struct Params {
   const float2* coef;  // [N] (g (1 - s), -g s): the gradient's two values per q (pass 2)
   float4* stats;       // [nchunk][N] (max_t, sum_t, max_d, sum_d), log2 units (pass 0)
   float2* partB;       // [nchunk][N] (a, s) (pass 1)
+  uint4* bits;         // [nvt][N] [q < p] of the tile's 128 entries (pass 1 writes, pass 2 reads)
   void* grad;          // [N][V] (pass 2)
 };
 
@@ -122,7 +124,13 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
   // 128-byte swizzled slices need 1024-byte aligned shared memory (the
   // dynamic region starts at the CTA's shared-memory base).
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  Hdr* hdr = reinterpret_cast<Hdr*>(smem_raw + kStages * kStageBytes);
+  // Passes 0 and 1 stage both models (rows and head of each: 64 KB, 3
+  // stages); pass 2 forms the draft logits only (32 KB, 6 stages): its
+  // [q < p] decisions come from pass 1.
+  constexpr int NM = MODE == 2 ? 1 : 2;
+  constexpr int kStageBytes = NM * 2 * kTile;
+  constexpr int kStages = kRing / kStageBytes;
+  Hdr* hdr = reinterpret_cast<Hdr*>(smem_raw + kRing);
   if (smem_u32(smem_raw) & 1023u) {  // uniform over the CTA; nothing touched yet
     if (threadIdx.x == 0) set_status(SPECOPD_DEV_LAYOUT);
     return;
@@ -175,10 +183,13 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
           }
           uint8_t* base = smem_raw + st * kStageBytes;
           mbar_arrive_expect_tx(&hdr->full[st], (unsigned)kStageBytes);
-          tma_load_2d(base, &tm_ht, kb * kBK, m * kBM, &hdr->full[st]);
-          tma_load_2d(base + kTile, &tm_wt, kb * kBK, vt * kBN, &hdr->full[st]);
-          tma_load_2d(base + 2 * kTile, &tm_hd, kb * kBK, m * kBM, &hdr->full[st]);
-          tma_load_2d(base + 3 * kTile, &tm_wd, kb * kBK, vt * kBN, &hdr->full[st]);
+          if constexpr (NM == 2) {
+            tma_load_2d(base, &tm_ht, kb * kBK, m * kBM, &hdr->full[st]);
+            tma_load_2d(base + kTile, &tm_wt, kb * kBK, vt * kBN, &hdr->full[st]);
+          }
+          uint8_t* bd = base + (NM - 1) * 2 * kTile;
+          tma_load_2d(bd, &tm_hd, kb * kBK, m * kBM, &hdr->full[st]);
+          tma_load_2d(bd + kTile, &tm_wd, kb * kBK, vt * kBN, &hdr->full[st]);
           ++q;
         }
       }
@@ -210,14 +221,15 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
           }
           tc_fence_after();
           const uint32_t base = smem_u32(smem_raw + st * kStageBytes);
+          const uint32_t bd = base + (NM - 1) * 2 * kTile;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             // K-major slices: 16 columns = 32 B inside each 128-byte swizzled row
             const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-            mma_ss(tT, sdesc(base + kk * 32, 16, 1024), sdesc(base + kTile + kk * 32, 16, 1024),
-                   kId, acc);
-            mma_ss(tD, sdesc(base + 2 * kTile + kk * 32, 16, 1024),
-                   sdesc(base + 3 * kTile + kk * 32, 16, 1024), kId, acc);
+            if constexpr (NM == 2)
+              mma_ss(tT, sdesc(base + kk * 32, 16, 1024), sdesc(base + kTile + kk * 32, 16, 1024),
+                     kId, acc);
+            mma_ss(tD, sdesc(bd + kk * 32, 16, 1024), sdesc(bd + kTile + kk * 32, 16, 1024), kId, acc);
           }
           tc_commit(&hdr->empty[st]);
           ++q;
@@ -255,10 +267,14 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
       tc_fence_after();
       __syncwarp();
       const uint32_t tT = tmem + lane_off + b * 2 * kBN, tD = tT + kBN;
+      // pass 1 writes, pass 2 reads the tile's [q < p] bits: word ch holds
+      // entries 32 ch .. 32 ch + 31 of the row
+      uint4 bw = make_uint4(0u, 0u, 0u, 0u);
+      if (MODE == 2 && row) bw = P.bits[(size_t)vt * P.N + n];
 #pragma unroll 1
       for (int ch = 0; ch < kBN / 32; ++ch) {
         uint32_t xt[32], xd[32];
-        tmem_ld32(tT + ch * 32, xt);
+        if constexpr (NM == 2) tmem_ld32(tT + ch * 32, xt);
         tmem_ld32(tD + ch * 32, xd);
         tmem_wait_ld();
         if (ch == kBN / 32 - 1) {
@@ -298,6 +314,7 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
           sT += at;
           sD += ad;
         } else if constexpr (MODE == 1) {
+          uint32_t mask = 0u;
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             if (e < nv) {
@@ -306,14 +323,16 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
               const float w = ex2_fast(fminf(lt, ld));
               pa += w;
               ps += (ld < lt) ? w : 0.f;
+              mask |= (ld < lt ? 1u : 0u) << e;
             }
+          if (ch == 0) bw.x = mask; else if (ch == 1) bw.y = mask; else if (ch == 2) bw.z = mask; else bw.w = mask;
         } else {
+          const uint32_t mask = ch == 0 ? bw.x : ch == 1 ? bw.y : ch == 2 ? bw.z : bw.w;
           float o[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float lt = fmaf(__uint_as_float(xt[e]), kLog2e, -Lt);
             const float ld = fmaf(__uint_as_float(xd[e]), kLog2e, -Ld);
-            o[e] = ex2_fast(ld) * ((ld < lt) ? c1 : c0);
+            o[e] = ex2_fast(ld) * (((mask >> e) & 1u) ? c1 : c0);
           }
           if (row) {
             Tg* dst = reinterpret_cast<Tg*>(P.grad) + (long long)n * P.V + v0;
@@ -341,6 +360,7 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
           }
         }
       }
+      if (MODE == 1 && row) P.bits[(size_t)vt * P.N + n] = bw;
     }
     if (row) {
       const float qnan = __int_as_float(0x7fc00000);
@@ -494,7 +514,7 @@ Plan make_plan(int N, int V, int nsm) {
 }
 
 struct Layout {
-  size_t ht, stats, lse, partB, coef, bsum, total;
+  size_t ht, stats, lse, partB, bits, coef, bsum, total;
 };
 
 Layout layout(const LmtvProblem& p, const Plan& pl) {
@@ -505,6 +525,7 @@ Layout layout(const LmtvProblem& p, const Plan& pl) {
   L.stats = off; off = up(off + sizeof(float4) * (size_t)pl.nchunk * p.N);
   L.lse = off;   off = up(off + sizeof(float2) * (size_t)p.N);
   L.partB = off; off = up(off + sizeof(float2) * (size_t)pl.nchunk * p.N);
+  L.bits = off;  off = up(off + sizeof(uint4) * (size_t)pl.nvt * p.N);
   L.coef = off;  off = up(off + sizeof(float2) * (size_t)p.N);
   L.bsum = off;  off = up(off + sizeof(double) * (size_t)p.nbranch);
   L.total = off;
@@ -525,7 +546,7 @@ bool make_map2d(CUtensorMap* m, const void* ptr, int cols, long long rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kSmem = (size_t)kStages * kStageBytes + sizeof(Hdr);
+constexpr size_t kSmem = (size_t)kRing + sizeof(Hdr);
 
 template <int MODE, typename Tg>
 cudaError_t launch_pass(const CUtensorMap* maps, const Params& P, int grid, cudaStream_t st) {
@@ -565,6 +586,7 @@ cudaError_t launch_lmtv(const LmtvProblem& p, const void* h_target, const int32_
   P.coef = reinterpret_cast<const float2*>(w + L.coef);
   P.stats = reinterpret_cast<float4*>(w + L.stats);
   P.partB = reinterpret_cast<float2*>(w + L.partB);
+  P.bits = reinterpret_cast<uint4*>(w + L.bits);
   P.grad = grad;
   const int grid = pl.mtiles * pl.nchunk;
   const long long nvec = (long long)p.N * (p.d / 8);
