@@ -776,10 +776,21 @@ def main():
                     help="skip the device-timed secondary workloads of the default run")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOAD_NAMES),
                     help="synthetic configuration (default: the 8B-shaped one)")
+    ap.add_argument("--lmhead-only", action="store_true",
+                    help="time only specopd_e2e_tv_lmhead (the LM heads fused in front of "
+                         "E2E-TV) and print its JSON object")
+    ap.add_argument("--lmhead-vocab", type=int, default=151936,
+                    help="vocabulary of the --lmhead-only run (smaller for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.lmhead_only:
+        import torch
+        from tree_attention_specopd_b200 import api
+        res = measure_lmhead_tv(torch, api, torch.device("cuda", 0), V=args.lmhead_vocab,
+                                reps=args.steps, warmup=args.warmup)
+        print(json.dumps(res), flush=True)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

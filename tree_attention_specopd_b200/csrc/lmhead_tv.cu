@@ -27,9 +27,9 @@
 //           gradient's mask are the same decisions).
 //  * Warp 0 drives TMA: per stage a 64-column slice (one 128-byte swizzled
 //    row) of the 128 target rows, of 128 rows of the target head, of the
-//    128 draft rows and of the draft head (4 x 16 KB, 3 stages; pass 2: the
-//    draft's two, 6 stages).  Rows past N or V and columns past d arrive as
-//    zeros.
+//    128 draft rows and of the draft head (4 x 16 KB, 3 stages; pass 2: two
+//    consecutive slices of the draft's rows and head).  Rows past N or V and
+//    columns past d arrive as zeros.
 //  * Warp 1 issues tcgen05.mma (M = N = 128, K = 16, both operands K-major
 //    from shared memory) from one thread, commits each stage back to the
 //    producer and each finished tile to the epilogue.
@@ -124,11 +124,14 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
   // 128-byte swizzled slices need 1024-byte aligned shared memory (the
   // dynamic region starts at the CTA's shared-memory base).
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // Passes 0 and 1 stage both models (rows and head of each: 64 KB, 3
-  // stages); pass 2 forms the draft logits only (32 KB, 6 stages): its
-  // [q < p] decisions come from pass 1.
-  constexpr int NM = MODE == 2 ? 1 : 2;
-  constexpr int kStageBytes = NM * 2 * kTile;
+  // A stage is 64 KB, 8 MMAs: passes 0 and 1 stage one 64-column slice of
+  // both models (rows and head of each), pass 2 two consecutive slices of
+  // the draft only (its [q < p] decisions come from pass 1).  Stages of 4
+  // MMAs (one model per stage, 32 KB) were measured slower: the cost per
+  // stage, not the copy latency, sets the rate.
+  constexpr int NM = MODE == 2 ? 1 : 2;  // models formed
+  constexpr int KPS = 3 - NM;            // 64-column slices per stage
+  constexpr int kStageBytes = 4 * kTile;
   constexpr int kStages = kRing / kStageBytes;
   Hdr* hdr = reinterpret_cast<Hdr*>(smem_raw + kRing);
   if (smem_u32(smem_raw) & 1023u) {  // uniform over the CTA; nothing touched yet
@@ -174,7 +177,7 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
       unsigned q = 0;  // stage sequence number
       bool live = true;
       for (int vt = vt0; vt < vt1 && live; ++vt) {
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = 0; kb < nkb; kb += KPS) {
           const int st = (int)(q % kStages);
           const unsigned use = q / kStages;
           if (use > 0u && !wait_or_abort(&hdr->empty[st], (use - 1u) & 1u, hdr)) {
@@ -182,14 +185,21 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
             break;
           }
           uint8_t* base = smem_raw + st * kStageBytes;
-          mbar_arrive_expect_tx(&hdr->full[st], (unsigned)kStageBytes);
           if constexpr (NM == 2) {
+            mbar_arrive_expect_tx(&hdr->full[st], (unsigned)kStageBytes);
             tma_load_2d(base, &tm_ht, kb * kBK, m * kBM, &hdr->full[st]);
             tma_load_2d(base + kTile, &tm_wt, kb * kBK, vt * kBN, &hdr->full[st]);
+            tma_load_2d(base + 2 * kTile, &tm_hd, kb * kBK, m * kBM, &hdr->full[st]);
+            tma_load_2d(base + 3 * kTile, &tm_wd, kb * kBK, vt * kBN, &hdr->full[st]);
+          } else {
+            const int nsub = min(2, nkb - kb);  // the last stage may hold one slice
+            mbar_arrive_expect_tx(&hdr->full[st], (unsigned)(nsub * 2 * kTile));
+            for (int sub = 0; sub < nsub; ++sub) {
+              tma_load_2d(base + sub * 2 * kTile, &tm_hd, (kb + sub) * kBK, m * kBM, &hdr->full[st]);
+              tma_load_2d(base + sub * 2 * kTile + kTile, &tm_wd, (kb + sub) * kBK, vt * kBN,
+                          &hdr->full[st]);
+            }
           }
-          uint8_t* bd = base + (NM - 1) * 2 * kTile;
-          tma_load_2d(bd, &tm_hd, kb * kBK, m * kBM, &hdr->full[st]);
-          tma_load_2d(bd + kTile, &tm_wd, kb * kBK, vt * kBN, &hdr->full[st]);
           ++q;
         }
       }
@@ -213,7 +223,7 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
         }
         tc_fence_after();
         const uint32_t tT = tmem + b * 2 * kBN, tD = tT + kBN;
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = 0; kb < nkb; kb += KPS) {
           const int st = (int)(q % kStages);
           if (!wait_or_abort(&hdr->full[st], (q / kStages) & 1u, hdr)) {
             ok = false;
@@ -221,15 +231,27 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
           }
           tc_fence_after();
           const uint32_t base = smem_u32(smem_raw + st * kStageBytes);
-          const uint32_t bd = base + (NM - 1) * 2 * kTile;
+          // K-major slices: 16 columns = 32 B inside each 128-byte swizzled row
+          if constexpr (NM == 2) {
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            // K-major slices: 16 columns = 32 B inside each 128-byte swizzled row
-            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-            if constexpr (NM == 2)
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
               mma_ss(tT, sdesc(base + kk * 32, 16, 1024), sdesc(base + kTile + kk * 32, 16, 1024),
                      kId, acc);
-            mma_ss(tD, sdesc(bd + kk * 32, 16, 1024), sdesc(bd + kTile + kk * 32, 16, 1024), kId, acc);
+              mma_ss(tD, sdesc(base + 2 * kTile + kk * 32, 16, 1024),
+                     sdesc(base + 3 * kTile + kk * 32, 16, 1024), kId, acc);
+            }
+          } else {
+            const int nsub = min(2, nkb - kb);
+            for (int sub = 0; sub < nsub; ++sub) {
+              const uint32_t bs = base + sub * 2 * kTile;
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk) {
+                const uint32_t acc = (kb + sub > 0 || kk > 0) ? 1u : 0u;
+                mma_ss(tD, sdesc(bs + kk * 32, 16, 1024), sdesc(bs + kTile + kk * 32, 16, 1024),
+                       kId, acc);
+              }
+            }
           }
           tc_commit(&hdr->empty[st]);
           ++q;
