@@ -28,8 +28,10 @@
 // so part of pass B's and pass C's re-reads come from DRAM.
 //
 // Roles: one producer warp issues the 1-D bulk copies (TMA) of every chunk
-// ahead of the consumers (pass A at normal L2 priority, pass B evict-last,
-// pass C evict-first); 12 consumer warps do the arithmetic; one scorer warp
+// ahead of the consumers (pass A at normal L2 priority, pass B evict-last
+// for what pass C reads again -- the draft row only when pass B keeps the
+// bits -- and evict-first otherwise, pass C evict-first); 12 consumer warps
+// do the arithmetic; one scorer warp
 // publishes each task's (a_n, s_n) from the consumer warps' partials, waits
 // for the branch, computes g_n and the owner's outputs, and hands g_n to the
 // consumers through an mbarrier.
@@ -191,11 +193,15 @@ __global__ void __launch_bounds__(tvrow::kThreads, 2) e2e_tv_row_kernel(const tv
       const uint64_t load = l2_policy_evict_normal();     // pass A
       const uint64_t keep = l2_policy_evict_last_full();  // pass B: read again by pass C
       const uint64_t drop = l2_policy_evict_first();      // pass C: last use
+      // With the [q < p] bits pass C reads the draft row only: pass B keeps
+      // just the draft in L2 (one row of one model per CTA, about 90 MB over
+      // the grid, which fits where both rows did not).
+      const uint64_t keep_t = A.bits ? drop : keep;
       const Tin* zt = reinterpret_cast<const Tin*>(A.zt);
       const Tin* zd = reinterpret_cast<const Tin*>(A.zd);
       unsigned q = 0;  // chunk sequence number over all tasks and passes (mod 2^32)
       bool live = true;
-      auto issue = [&](const Tin* rt, const Tin* rd, int c, uint64_t pol) {
+      auto issue = [&](const Tin* rt, const Tin* rd, int c, uint64_t pol_t, uint64_t pol) {
         if (!live) return;
         const int st = (int)(q % kStages);
         const unsigned use = q / kStages;
@@ -208,7 +214,7 @@ __global__ void __launch_bounds__(tvrow::kThreads, 2) e2e_tv_row_kernel(const tv
         const unsigned bytes = (unsigned)(min(CE, V - e0) * (int)sizeof(Tin));
         uint8_t* dst = ring + (size_t)st * 2 * kChunkBytes;
         mbar_arrive_expect_tx(&sh.full[st], 2u * bytes);
-        bulk_g2s_hint(dst, rt + e0, bytes, &sh.full[st], pol);
+        bulk_g2s_hint(dst, rt + e0, bytes, &sh.full[st], pol_t);
         bulk_g2s_hint(dst + kChunkBytes, rd + e0, bytes, &sh.full[st], pol);
         ++q;
       };
@@ -243,12 +249,12 @@ __global__ void __launch_bounds__(tvrow::kThreads, 2) e2e_tv_row_kernel(const tv
         }
         for (int i = -kLag; i < nch; ++i) {
           if (hasC && i >= 0) {
-            if (A.bits) issue_d(rd_prev, i, drop); else issue(rt_prev, rd_prev, i, drop);
+            if (A.bits) issue_d(rd_prev, i, drop); else issue(rt_prev, rd_prev, i, drop, drop);
           }
-          if (hasA && i + kLag < nch) issue(rt, rd, i + kLag, load);
+          if (hasA && i + kLag < nch) issue(rt, rd, i + kLag, load, load);
         }
         if (hasA)
-          for (int c = 0; c < nch; ++c) issue(rt, rd, c, keep);
+          for (int c = 0; c < nch; ++c) issue(rt, rd, c, keep_t, keep);
         rt_prev = rt;
         rd_prev = rd;
       }
