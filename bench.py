@@ -473,9 +473,9 @@ def measure_lmhead_tv(torch, api, dev, nbranch=64, W=8, V=151936, d=4096, reps=5
     """Device time of specopd_e2e_tv_lmhead (the LM heads fused in front of
     E2E-TV) on the 8B shape with a 4096-wide hidden state: seeded bf16 hidden
     rows and heads made on the device with the synth recipe's distributions,
-    CUDA events around `reps` calls after `warmup`.  Executed tensor work:
-    passes 0 and 1 form both models' logits, pass 2 the draft's (5 GEMMs of
-    2 N V d FLOPs)."""
+    CUDA events around `reps` calls after `warmup`.  Executed tensor work
+    with the fp32 gradient: passes 0 and 1 form both models' logits (4 GEMMs
+    of 2 N V d FLOPs); the gradient is then scaled in place."""
     N = nbranch * W
     g = torch.Generator(device=dev)
     g.manual_seed(1234)
@@ -504,7 +504,7 @@ def measure_lmhead_tv(torch, api, dev, nbranch=64, W=8, V=151936, d=4096, reps=5
     if st != 0:
         raise RuntimeError(f"device status {st:#x} after specopd_e2e_tv_lmhead")
     ms = e0.elapsed_time(e1) / reps
-    flops = 5 * 2.0 * N * V * d
+    flops = 4 * 2.0 * N * V * d
     peaks = _peaks()
     tf = flops / (ms / 1e3) / 1e12
     res = {"call": "specopd_e2e_tv_lmhead", "nbranch": nbranch, "W": W, "V": V, "d_model": d,

@@ -21,10 +21,15 @@
 //   pass 1: per row, sum_v 2^min(lt, ld) and the [ld < lt] part of it over
 //           the chunk -> one (a, s) record per (chunk, row);
 //   (branch: a_n, s_n in chunk order, prefix products, g_n, the loss)
-//   pass 1 also stores [q_v < p_v] of every entry (one bit; N V / 8 bytes);
-//   pass 2: the draft tiles only, dz_d[n, v] = g_n q_v ([q_v < p_v] - s_n)
-//           with pass 1's bits, written as the tile's epilogue (so s_n and the
-//           gradient's mask are the same decisions).
+//   then the gradient dz_d[n, v] = g_n q_v ([q_v < p_v] - s_n), whose two
+//   values per row, g (1 - s) and -g s, are known only after the branch:
+//   - fp32 gradient: pass 1 (as MODE 3) writes q_v into the gradient row with
+//     [q_v < p_v] in its sign, and an elementwise kernel multiplies in place
+//     (four GEMMs per call);
+//   - bf16 gradient: pass 1 stores [q_v < p_v] as one bit (N V / 8 bytes) and
+//     pass 2 forms the draft tiles again and writes the gradient as its
+//     epilogue (a rounded q would be rounded twice).
+//   Either way s_n and the gradient's mask are the same decisions.
 //  * Warp 0 drives TMA: per stage a 64-column slice (one 128-byte swizzled
 //    row) of the 128 target rows, of 128 rows of the target head, of the
 //    128 draft rows and of the draft head (4 x 16 KB, 3 stages; pass 2: two
@@ -115,7 +120,10 @@ __device__ __forceinline__ void chunk_tiles(const Params& P, int c, int& vt0, in
 }
 
 // One pass over the CTA's (row tile, vocabulary chunk): MODE 0 statistics,
-// 1 overlap partials, 2 gradient tiles (Tg = the gradient's element type).
+// 1 overlap partials and the [q < p] bits, 2 gradient tiles from the bits
+// (Tg = the gradient's element type), 3 overlap partials and, for an fp32
+// gradient, q_v written in place with [q_v < p_v] in its sign (negative:
+// false), which lmtv_scale_kernel turns into the gradient.
 template <int MODE, typename Tg>
 __global__ void __launch_bounds__(kThreads, 1)
 lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ CUtensorMap tm_wt,
@@ -335,10 +343,12 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
             }
           sT += at;
           sD += ad;
-        } else if constexpr (MODE == 1) {
+        } else if constexpr (MODE == 1 || MODE == 3) {
           uint32_t mask = 0u;
+          float o[32];  // pass 3: q_v, negated where [q_v < p_v] is false
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
+          for (int e = 0; e < 32; ++e) {
+            o[e] = 0.f;
             if (e < nv) {
               const float lt = fmaf(__uint_as_float(xt[e]), kLog2e, -Lt);
               const float ld = fmaf(__uint_as_float(xd[e]), kLog2e, -Ld);
@@ -346,8 +356,23 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
               pa += w;
               ps += (ld < lt) ? w : 0.f;
               mask |= (ld < lt ? 1u : 0u) << e;
+              if constexpr (MODE == 3) o[e] = (ld < lt) ? w : -ex2_fast(ld);
             }
-          if (ch == 0) bw.x = mask; else if (ch == 1) bw.y = mask; else if (ch == 2) bw.z = mask; else bw.w = mask;
+          }
+          if constexpr (MODE == 1) {
+            if (ch == 0) bw.x = mask; else if (ch == 1) bw.y = mask; else if (ch == 2) bw.z = mask; else bw.w = mask;
+          } else if (row) {
+            float* dst = reinterpret_cast<float*>(P.grad) + (long long)n * P.V + v0;
+            if (nv == 32) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (e < nv) dst[e] = o[e];
+            }
+          }
         } else {
           const uint32_t mask = ch == 0 ? bw.x : ch == 1 ? bw.y : ch == 2 ? bw.z : bw.w;
           float o[32];
@@ -388,7 +413,7 @@ lmtv_kernel(const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ C
       const float qnan = __int_as_float(0x7fc00000);
       if constexpr (MODE == 0)
         P.stats[(size_t)c * P.N + n] = dead ? make_float4(qnan, qnan, qnan, qnan) : make_float4(mt, sT, md, sD);
-      if constexpr (MODE == 1)
+      if constexpr (MODE == 1 || MODE == 3)
         P.partB[(size_t)c * P.N + n] = dead ? make_float2(qnan, qnan) : make_float2(pa, ps);
     }
   }
@@ -480,6 +505,24 @@ __global__ void lmtv_branch_kernel(const float2* partB, int nchunk, int N, int n
     sumP += (double)P;
   }
   bsum[b] = sumP;
+}
+
+// fp32 gradient in place from pass 3's signed q_v: dz = |v| * (v >= 0 ? c1 : c0)
+// with (c1, c0) = (g (1 - s), -g s) of its row; the same product pass 2 forms.
+// Columns in float4 (V % 4 == 0), rows strided over gridDim.y.
+__global__ void lmtv_scale_kernel(float* grad, const float2* coef, int N, int V) {
+  const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c4 >= V / 4) return;
+  for (int n = blockIdx.y; n < N; n += gridDim.y) {
+    float4* p = reinterpret_cast<float4*>(grad + (size_t)n * V) + c4;
+    const float2 cf = coef[n];
+    float4 v = __ldcs(p);
+    v.x = fabsf(v.x) * (signbit(v.x) ? cf.y : cf.x);
+    v.y = fabsf(v.y) * (signbit(v.y) ? cf.y : cf.x);
+    v.z = fabsf(v.z) * (signbit(v.z) ? cf.y : cf.x);
+    v.w = fabsf(v.w) * (signbit(v.w) ? cf.y : cf.x);
+    __stcs(p, v);
+  }
 }
 
 // loss = 1 - sum_b bsum[b] / norm, in a fixed summation order (one block).
@@ -621,7 +664,13 @@ cudaError_t launch_lmtv(const LmtvProblem& p, const void* h_target, const int32_
   lmtv_stats_kernel<<<(p.N + 255) / 256, 256, 0, st>>>(P.stats, pl.nchunk, p.N, target_row,
                                                        p.rows_target, reinterpret_cast<float2*>(w + L.lse));
   e = cudaGetLastError();
-  if (e == cudaSuccess) e = launch_pass<1, float>(maps, P, grid, st);
+  // An fp32 gradient is formed in place: pass 3 writes q_v with its [q < p]
+  // sign, the scale kernel applies the row's two values once g_n is known.
+  // A bf16 gradient needs pass 1's bits and pass 2 (a rounded q would be
+  // rounded twice).
+  const bool inplace = p.compute_grad && grad && p.grad_dtype == SPECOPD_F32;
+  if (e == cudaSuccess) e = inplace ? launch_pass<3, float>(maps, P, grid, st)
+                                    : launch_pass<1, float>(maps, P, grid, st);
   if (e != cudaSuccess) return e;
   lmtv_branch_kernel<<<(p.nbranch + 127) / 128, 128, 0, st>>>(
       P.partB, pl.nchunk, p.N, p.nbranch, p.W, P.lse, (float)(1.0 / p.norm_count), a, prefix,
@@ -630,8 +679,12 @@ cudaError_t launch_lmtv(const LmtvProblem& p, const void* h_target, const int32_
                                       p.norm_count, loss, numer);
   e = cudaGetLastError();
   if (e != cudaSuccess || !p.compute_grad || !grad) return e;
-  return p.grad_dtype == SPECOPD_BF16 ? launch_pass<2, __nv_bfloat16>(maps, P, grid, st)
-                                      : launch_pass<2, float>(maps, P, grid, st);
+  if (inplace) {
+    const dim3 sg((unsigned)((p.V / 4 + 255) / 256), (unsigned)std::min(p.N, 64));
+    lmtv_scale_kernel<<<sg, 256, 0, st>>>(reinterpret_cast<float*>(grad), P.coef, p.N, p.V);
+    return cudaGetLastError();
+  }
+  return launch_pass<2, __nv_bfloat16>(maps, P, grid, st);
 }
 
 }  // namespace specopd
