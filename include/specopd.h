@@ -326,8 +326,9 @@ specopd_status specopd_e2e_tv_finalize(const double* numer_sum, int64_t norm_cou
  *   z_t[n] = W_target h_target[target_row[n]],   z_d[n] = W_draft h_draft[n]
  * (fp32 accumulation of bf16 products; no bias, norm or temperature), then
  * a, prefix, numer, loss and grad_draft = d loss / d z_d exactly as
- * specopd_e2e_tv defines them.  Three passes over the heads (statistics,
- * overlaps, gradient), each reading both heads once.
+ * specopd_e2e_tv defines them.  Two passes over both heads (statistics,
+ * overlaps); an fp32 gradient is then finished in place by one elementwise
+ * pass, a bf16 gradient by a third pass over the draft head.
  */
 typedef struct {
   int nbranch;               /* S*B branches                                 */
@@ -336,7 +337,7 @@ typedef struct {
   int d_model;               /* hidden size, a multiple of 8                 */
   int rows_target;           /* rows of h_target (bounds for target_row)     */
   specopd_dtype grad_dtype;  /* grad_draft                                   */
-  int compute_grad;          /* 0: skip grad_draft (two passes instead of 3) */
+  int compute_grad;          /* 0: skip grad_draft                           */
   int64_t norm_count;        /* divisor of the loss; 0 -> nbranch*W          */
 } specopd_lmhead_tv_desc;
 
