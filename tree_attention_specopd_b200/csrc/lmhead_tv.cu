@@ -11,8 +11,8 @@
 //   z_t[n] = W_t h_t[target_row[n]],   z_d[n] = W_d h_d[n]      (fp32 accumulation)
 //   then a_n, prefix products, loss and dz_d exactly as specopd_e2e_tv.
 //
-// B200 design.  Three passes of one tcgen05 GEMM kernel over tiles of 128
-// positions x 128 vocabulary entries, each tile holding both models'
+// B200 design.  Two or three passes of one tcgen05 GEMM kernel over tiles of
+// 128 positions x 128 vocabulary entries, each tile holding both models'
 // logits in TMEM (fp32, 2 x 128 columns, double-buffered: 512 columns, one
 // CTA per SM; pass 2 the draft's only), with a per-pass epilogue:
 //   pass 0: per row, running (max, sum of 2^(x - max)) of both rows over the
