@@ -9,7 +9,9 @@ position count, so its gradient already carries the global 1/N), the ranks
 all-reduce their `numer` outputs, and specopd_e2e_tv_finalize writes the
 loss on the device.  Every rank's overlaps, prefix products and gradient rows
 and the common loss must match the single-process fp64 oracle, also when the
-ranks hold different numbers of branches.
+ranks hold different numbers of branches.  The same holds for the call with
+the LM heads fused in front (specopd_e2e_tv_lmhead), each rank holding the
+hidden rows of its own positions.
 """
 
 import os
@@ -21,6 +23,7 @@ import torch
 import torch.multiprocessing as mp
 
 import synth
+from oracle import lmhead as olm
 from oracle import tv as otv
 
 pytestmark = pytest.mark.gpu
@@ -41,7 +44,11 @@ def _data(nb, W, V):
     return synth.round_bf16(zt), synth.round_bf16(zd)
 
 
-def _rank(rank, world, port, nb, W, V, out_q):
+def _lm_data(nb, W, V):
+    return synth.lmhead_inputs(nb * 100 + W, nb, W, V, 128)
+
+
+def _rank(rank, world, port, nb, W, V, out_q, fused=False):
     import datetime
 
     import torch.distributed as dist
@@ -59,8 +66,16 @@ def _rank(rank, world, port, nb, W, V, out_q):
         rows = slice(start * W, (start + cnt) * W)
         n_global = sdist.global_count(cnt * W)
         t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to("cuda").to(torch.bfloat16)  # noqa
-        desc = api.tv_desc(cnt, W, V, cnt * W, "bf16", "f32", True, norm_count=n_global)
-        res = api.specopd_e2e_tv(desc, t(zt[rows]), None, t(zd[rows]))
+        if fused:
+            x = _lm_data(nb, W, V)
+            ht = x.h_target[x.target_row[rows]]  # this rank's scoring rows, in position order
+            desc = api.lmhead_tv_desc(cnt, W, V, x.w_target.shape[1], cnt * W, "f32", True,
+                                      norm_count=n_global)
+            res = api.specopd_e2e_tv_lmhead(desc, t(ht), None, t(x.w_target), t(x.h_draft[rows]),
+                                            t(x.w_draft))
+        else:
+            desc = api.tv_desc(cnt, W, V, cnt * W, "bf16", "f32", True, norm_count=n_global)
+            res = api.specopd_e2e_tv(desc, t(zt[rows]), None, t(zd[rows]))
         loss = sdist.global_loss(res["numer"], n_global)
         torch.cuda.synchronize()
         status = api.specopd_get_device_status()
@@ -70,21 +85,30 @@ def _rank(rank, world, port, nb, W, V, out_q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("nb", [10, 11])  # 11: the ranks hold 6 and 5 branches
-def test_two_ranks_through_the_library(lib, nb):
+@pytest.mark.parametrize("nb,fused", [(10, False), (11, False), (11, True)])  # 11: 6 and 5 branches
+def test_two_ranks_through_the_library(lib, nb, fused):
     W, V, world = 4, 4096, 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, nb, W, V, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, nb, W, V, q, fused))
+             for r in range(world)]
     for p in procs:
         p.start()
     results = [q.get(timeout=300) for _ in range(world)]
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
-    zt, zd = _data(nb, W, V)
-    full = otv.e2e_tv(zt, None, zd, nb, W)
+    if fused:
+        x = _lm_data(nb, W, V)
+        full = olm.e2e_tv_lmhead(x.h_target, x.target_row, x.w_target, x.h_draft, x.w_draft, nb, W)
+        # logits formed on the tensor cores (fp32 sums of 128 bf16 products):
+        # the fused call's bound, 1e-5 + 2 sqrt(d) 2^-24 zmax with zmax < 40
+        rtol = 1e-5 + 2.0 * np.sqrt(128) * 2.0 ** -24 * 40.0
+    else:
+        zt, zd = _data(nb, W, V)
+        full = otv.e2e_tv(zt, None, zd, nb, W)
+        rtol = 1e-5
     for rank, start, cnt, n_global, loss, a, prefix, grad, status in results:
         assert status == 0
         assert n_global == nb * W
@@ -92,8 +116,8 @@ def test_two_ranks_through_the_library(lib, nb):
         rows = range(start * W, (start + cnt) * W)
         ref_a = full["a"][start * W:(start + cnt) * W]
         ref_p = full["prefix"][start * W:(start + cnt) * W]
-        assert np.all(np.abs(a - ref_a) <= 1e-5 * np.abs(ref_a) + 1e-7)
-        assert np.all(np.abs(prefix - ref_p) <= 1e-5 * np.abs(ref_p) + 1e-7)
+        assert np.all(np.abs(a - ref_a) <= rtol * np.abs(ref_a) + 1e-7)
+        assert np.all(np.abs(prefix - ref_p) <= rtol * np.abs(ref_p) + 1e-7)
         for k, n in enumerate(rows):
             gr = full["grad"][n]
             err = np.max(np.abs(grad[k] - gr)) / np.max(np.abs(gr))
