@@ -669,6 +669,9 @@ cudaError_t launch_lmtv(const LmtvProblem& p, const void* h_target, const int32_
   // A bf16 gradient needs pass 1's bits and pass 2 (a rounded q would be
   // rounded twice).
   const bool inplace = p.compute_grad && grad && p.grad_dtype == SPECOPD_F32;
+  // the in-place path moves whole float4 of a row (16-byte aligned rows)
+  if (inplace && (p.V % 4 != 0 || reinterpret_cast<uintptr_t>(grad) % 16 != 0))
+    return cudaErrorInvalidValue;
   if (e == cudaSuccess) e = inplace ? launch_pass<3, float>(maps, P, grid, st)
                                     : launch_pass<1, float>(maps, P, grid, st);
   if (e != cudaSuccess) return e;
