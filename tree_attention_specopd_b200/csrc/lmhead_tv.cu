@@ -638,6 +638,13 @@ cudaError_t launch_lmtv(const LmtvProblem& p, const void* h_target, const int32_
   const Plan pl = make_plan(p.N, p.V, sm100::sm_count());
   const Layout L = layout(p, pl);
   if (ws_bytes < L.total) return cudaErrorInvalidValue;
+  // An fp32 gradient is formed in place: pass 3 writes q_v with its [q < p]
+  // sign, the scale kernel applies the row's two values once g_n is known.
+  // A bf16 gradient needs pass 1's bits and pass 2 (a rounded q would be
+  // rounded twice).  The in-place path moves whole float4 of a row.
+  const bool inplace = p.compute_grad && grad && p.grad_dtype == SPECOPD_F32;
+  if (inplace && (p.V % 4 != 0 || reinterpret_cast<uintptr_t>(grad) % 16 != 0))
+    return cudaErrorInvalidValue;
   char* w = reinterpret_cast<char*>(ws);
   void* ht = w + L.ht;
   CUtensorMap maps[4];
@@ -664,14 +671,6 @@ cudaError_t launch_lmtv(const LmtvProblem& p, const void* h_target, const int32_
   lmtv_stats_kernel<<<(p.N + 255) / 256, 256, 0, st>>>(P.stats, pl.nchunk, p.N, target_row,
                                                        p.rows_target, reinterpret_cast<float2*>(w + L.lse));
   e = cudaGetLastError();
-  // An fp32 gradient is formed in place: pass 3 writes q_v with its [q < p]
-  // sign, the scale kernel applies the row's two values once g_n is known.
-  // A bf16 gradient needs pass 1's bits and pass 2 (a rounded q would be
-  // rounded twice).
-  const bool inplace = p.compute_grad && grad && p.grad_dtype == SPECOPD_F32;
-  // the in-place path moves whole float4 of a row (16-byte aligned rows)
-  if (inplace && (p.V % 4 != 0 || reinterpret_cast<uintptr_t>(grad) % 16 != 0))
-    return cudaErrorInvalidValue;
   if (e == cudaSuccess) e = inplace ? launch_pass<3, float>(maps, P, grid, st)
                                     : launch_pass<1, float>(maps, P, grid, st);
   if (e != cudaSuccess) return e;
