@@ -443,21 +443,30 @@ __global__ void lmtv_gather_kernel(const uint4* h, const int32_t* trow, int rows
   out[i] = ok ? h[(long long)r * d8 + k] : make_uint4(0u, 0u, 0u, 0u);
 }
 
-// lse of both rows from the chunks' records, combined in chunk order.  A
-// row whose target row is out of range, or whose records carry a NaN (a wait
-// ran out), gets NaN.
+// lse of both rows from the chunks' records: one warp per row, lane l
+// combining chunks l, l + 32, ... in order, then a fixed butterfly over the
+// lanes (the same combination order on every call).  A row whose target row
+// is out of range, or whose records carry a NaN (a wait ran out), gets NaN.
 __global__ void lmtv_stats_kernel(const float4* stats, int nchunk, int N, const int32_t* trow,
                                   int rows_target, float2* lse) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
+  const int n = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (n >= N) return;  // uniform over the warp
   float mt = -INFINITY, st = 0.f, md = -INFINITY, sd = 0.f;
   bool bad = false;
-  for (int c = 0; c < nchunk; ++c) {
+  for (int c = lane; c < nchunk; c += 32) {
     const float4 r = stats[(size_t)c * N + n];
     bad |= isnan(r.x) || isnan(r.y) || isnan(r.z) || isnan(r.w);
     lse2_combine(mt, st, r.x, r.y);
     lse2_combine(md, sd, r.z, r.w);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lse2_combine(mt, st, __shfl_xor_sync(0xffffffffu, mt, o), __shfl_xor_sync(0xffffffffu, st, o));
+    lse2_combine(md, sd, __shfl_xor_sync(0xffffffffu, md, o), __shfl_xor_sync(0xffffffffu, sd, o));
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane != 0) return;
   const int row = trow ? trow[n] : n;
   const float qnan = __int_as_float(0x7fc00000);
   if (row < 0 || row >= rows_target || bad || mt == -INFINITY || md == -INFINITY) {
@@ -467,29 +476,34 @@ __global__ void lmtv_stats_kernel(const float4* stats, int nchunk, int N, const 
   }
 }
 
-// Per branch: a_n and s_n from the chunks' (a, s) records in chunk order,
-// the prefix products, g_n and the gradient's two values per q, and the
-// branch's sum of prefix products.  One thread per branch.
+// Per branch: a_n and s_n from the chunks' (a, s) records (one warp per
+// branch: lane l sums chunks l, l + 32, ... in order, then a fixed butterfly
+// over the lanes), then on lane 0 the prefix products, g_n and the
+// gradient's two values per q, and the branch's sum of prefix products.
 __global__ void lmtv_branch_kernel(const float2* partB, int nchunk, int N, int nbranch, int W,
                                    const float2* lse, float inv_norm, float* a_out, float* prefix,
                                    float2* coef, double* bsum) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= nbranch) return;
+  const int b = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (b >= nbranch) return;  // uniform over the warp
   const float qnan = __int_as_float(0x7fc00000);
   float sa[kMaxW], ss[kMaxW];
   for (int i = 0; i < W; ++i) {
     const int n = b * W + i;
     float a = 0.f, s = 0.f;
-    for (int c = 0; c < nchunk; ++c) {
+    for (int c = lane; c < nchunk; c += 32) {
       const float2 r = partB[(size_t)c * N + n];
       a += r.x;
       s += r.y;
     }
+    a = warp_sum(a);
+    s = warp_sum(s);
     const float2 L = lse[n];
     if (isnan(L.x) || isnan(L.y)) a = s = qnan;
     sa[i] = a;
     ss[i] = s;
   }
+  if (lane != 0) return;
   float P = 1.f;
   double sumP = 0.0;
   for (int i = 0; i < W; ++i) {
@@ -668,13 +682,13 @@ cudaError_t launch_lmtv(const LmtvProblem& p, const void* h_target, const int32_
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) e = launch_pass<0, float>(maps, P, grid, st);
   if (e != cudaSuccess) return e;
-  lmtv_stats_kernel<<<(p.N + 255) / 256, 256, 0, st>>>(P.stats, pl.nchunk, p.N, target_row,
+  lmtv_stats_kernel<<<(unsigned)(((size_t)p.N * 32 + 255) / 256), 256, 0, st>>>(P.stats, pl.nchunk, p.N, target_row,
                                                        p.rows_target, reinterpret_cast<float2*>(w + L.lse));
   e = cudaGetLastError();
   if (e == cudaSuccess) e = inplace ? launch_pass<3, float>(maps, P, grid, st)
                                     : launch_pass<1, float>(maps, P, grid, st);
   if (e != cudaSuccess) return e;
-  lmtv_branch_kernel<<<(p.nbranch + 127) / 128, 128, 0, st>>>(
+  lmtv_branch_kernel<<<(unsigned)(((size_t)p.nbranch * 32 + 127) / 128), 128, 0, st>>>(
       P.partB, pl.nchunk, p.N, p.nbranch, p.W, P.lse, (float)(1.0 / p.norm_count), a, prefix,
       reinterpret_cast<float2*>(w + L.coef), reinterpret_cast<double*>(w + L.bsum));
   lmtv_loss_kernel<<<1, 256, 0, st>>>(reinterpret_cast<const double*>(w + L.bsum), p.nbranch,
