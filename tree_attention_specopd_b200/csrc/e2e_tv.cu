@@ -697,7 +697,12 @@ cudaError_t launch_row(const TVProblem& p, bool aligned, const void* z_target,
   // Two CTAs per SM (the kernel's geometry).
   const long long resident = (long long)std::min(per_sm, 2) * nsm;
   if (p.W > resident) return cudaErrorNotSupported;
-  const long long G = resident / p.W * p.W;  // whole branches per round
+  // Whole branches per round, at most the resident CTAs; the rounds that
+  // takes are then spread evenly (N = 512 at 296 slots: two rounds of 256
+  // instead of 296 + 216; measured 180 against 184 us, bit-identical).
+  const long long G0 = resident / p.W * p.W;
+  const long long rounds = (p.N + G0 - 1) / G0;
+  const long long G = std::min(G0, ((p.N + rounds - 1) / rounds + p.W - 1) / p.W * p.W);
   const int grid = (int)std::min<long long>(G, p.N);
   // The ring's chunk counter is 32-bit: keep a CTA's chunks below 2^32.
   const long long ce = (long long)kConsumers * kVPT * (16 / elt_size(p.logit_dtype));
