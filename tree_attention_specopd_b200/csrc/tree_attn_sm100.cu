@@ -56,6 +56,10 @@ constexpr int kBN = 64;        // keys per tile
 constexpr int kKStages = 3;    // K ring depth (K tiles run ahead of V tiles)
 constexpr int kVStages = 2;    // V ring depth
 constexpr int kCtasPerSm = 2;
+// Key tiles that chunk 0 of a split (tile, kv head) pair is counted heavier
+// when its trunk keys are shared out (it also scores and rotates the branch
+// tiles and is usually the one that merges).
+constexpr int kChunk0Extra = 4;
 constexpr int kTmemCols = 256;              // S0 [0,64), S1 [64,128), O [128, 128+D)
 constexpr int kQHalf = 128 * 128;           // Q box: 128 rows x 64 bf16 (swizzled)
 constexpr int kKVHalf = kBN * 128;          // K/V box: 64 rows x 64 bf16 (swizzled)
@@ -68,6 +72,8 @@ struct Params {
   int RT;              // branch rows per query tile
   int ntile_per_seq, ntile;
   int nsplit, C;       // key chunks per (tile, kv head), keys per chunk (multiple of kBN)
+  int s_lo, n_hi;      // s_lo > 0: the heaviest n_hi tiles split in s_lo + 1 chunks, the
+                       // others in s_lo, each pair's chunks sized from its own key span
   float scale_log2;    // softmax scale * log2(e)
   const int32_t* cu_trunk;
   const int32_t* anchors;
@@ -299,10 +305,32 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   // first row, and row r sees the rows of its own sequence up to itself.
   // In both cases row r sees the keys t0 + vlo_r .. t0 + vhi_r.
   const int u = blockIdx.x;
-  const int per_c = P.ntile * P.Hkv;
-  const int c = u / per_c;
-  const int tile = P.ntile - 1 - (u % per_c) / P.Hkv;
-  const int h = (u % per_c) % P.Hkv;
+  int c, tile, h, nsp = 0;  // nsp > 0: this pair's chunk count (chunk size from its span)
+  if (P.s_lo > 0) {
+    // One wave of units: the n_hi heaviest tiles (the last ones) in s_lo + 1
+    // chunks, the others in s_lo; heavier tiles first within each group.
+    const int heavy = P.n_hi * P.Hkv;
+    const int u_hi = heavy * (P.s_lo + 1);
+    int rem;
+    if (u < u_hi) {
+      c = u / heavy;
+      rem = u % heavy;
+      tile = P.ntile - 1 - rem / P.Hkv;
+      nsp = P.s_lo + 1;
+    } else {
+      const int light = (P.ntile - P.n_hi) * P.Hkv;
+      c = (u - u_hi) / light;
+      rem = (u - u_hi) % light;
+      tile = P.ntile - P.n_hi - 1 - rem / P.Hkv;
+      nsp = P.s_lo;
+    }
+    h = rem % P.Hkv;
+  } else {
+    const int per_c = P.ntile * P.Hkv;
+    c = u / per_c;
+    tile = P.ntile - 1 - (u % per_c) / P.Hkv;
+    h = (u % per_c) % P.Hkv;
+  }
   const int Wm1 = P.W - 1;
   int s, r0, r1;
   if (P.prefill) {
@@ -386,9 +414,29 @@ tree_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = hdr->tmem_base;
   const int kmax = max(max(hdr->wmax[0], hdr->wmax[1]), max(hdr->wmax[2], hdr->wmax[3]));
-  const int nact = kmax < 0 ? 1 : (kmax + P.C) / P.C;  // chunks with trunk keys (>= 1)
-  const int k_begin = c * P.C;
-  const int k_end = min(k_begin + P.C, kmax + 1);
+  // Trunk keys of this chunk.  Fixed chunks of P.C keys, or (nsp > 0) this
+  // pair's key tiles split over its nsp chunks with chunk 0 -- which also
+  // scores and rotates the branch tiles and usually merges -- counted
+  // kChunk0Extra tiles heavier.  Either way the chunks that hold keys are
+  // 0 .. nact - 1, the same on every unit of the pair.
+  int nact, k_begin, k_end;
+  if (nsp > 0) {
+    const int ntk = kmax < 0 ? 0 : (kmax + 1 + kBN - 1) / kBN;  // trunk key tiles
+    int t0n = ntk, per = 1;  // trunk tiles of chunk 0, of the others
+    if (nsp > 1) {
+      t0n = min(ntk, max(0, (ntk + kChunk0Extra + nsp - 1) / nsp - kChunk0Extra));
+      per = max(1, (ntk - t0n + nsp - 2) / (nsp - 1));
+    }
+    nact = 1 + (ntk > t0n ? (ntk - t0n + per - 1) / per : 0);
+    const int tb = c == 0 ? 0 : t0n + (c - 1) * per;
+    const int te = c == 0 ? t0n : min(ntk, t0n + c * per);
+    k_begin = tb * kBN;
+    k_end = min(te * kBN, kmax + 1);
+  } else {
+    nact = kmax < 0 ? 1 : (kmax + P.C) / P.C;  // chunks with trunk keys (>= 1)
+    k_begin = c * P.C;
+    k_end = min(k_begin + P.C, kmax + 1);
+  }
   const int nt = k_end > k_begin ? (k_end - k_begin + kBN - 1) / kBN : 0;
   if (c > 0 && nt == 0) {
     // Nothing for this chunk (uniform over the CTA).  The Q copy must land
@@ -795,6 +843,8 @@ bool make_map(CUtensorMap* m, const void* ptr, int D, int H, int rows, int box_h
 
 struct Plan {
   int RT, ntile_per_seq, ntile, nsplit, C;
+  int s_lo, n_hi;  // one-wave split of the branch pass (s_lo > 0), see make_plan
+  long long units;
   size_t part_bytes, cnt_bytes;
 };
 
@@ -830,6 +880,23 @@ Plan make_plan(const AttnProblem& p, int num_sms, bool prefill) {
   C = (C + kBN - 1) / kBN * kBN;
   pl.nsplit = (key_span + C - 1) / C;
   pl.C = C;
+  pl.s_lo = 0;
+  pl.n_hi = 0;
+  pl.units = base * pl.nsplit;
+  if (!prefill && base < slots) {
+    // Fewer (tile, kv head) pairs than CTA slots: split so that the units
+    // fit one wave exactly -- s_lo chunks per pair, one more for the
+    // heaviest tiles while slots remain -- each pair's chunks sized on the
+    // device from its own key span.  A fixed chunk size left units for a
+    // second wave (8B: 304 of 336 non-empty on 296 slots).
+    const int cap = std::min(max_split, 64);
+    const int s_lo = (int)std::min<long long>(std::max<long long>(1, slots / base), cap);
+    const int n_hi = s_lo < cap ? (int)std::min<long long>(pl.ntile, (slots - base * s_lo) / p.Hkv) : 0;
+    pl.s_lo = s_lo;
+    pl.n_hi = n_hi;
+    pl.nsplit = s_lo + (n_hi > 0 ? 1 : 0);
+    pl.units = (long long)n_hi * p.Hkv * (s_lo + 1) + (long long)(pl.ntile - n_hi) * p.Hkv * s_lo;
+  }
   pl.part_bytes = pl.nsplit > 1 ? (size_t)pl.ntile * p.Hkv * pl.nsplit * ((size_t)128 * p.D + 256) * 4 : 0;
   pl.cnt_bytes = (size_t)pl.ntile * p.Hkv * 4;
   return pl;
@@ -887,6 +954,7 @@ cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_br, const void
   P.T_tot = p.T_tot;
   P.RT = pl.RT; P.ntile_per_seq = pl.ntile_per_seq; P.ntile = pl.ntile;
   P.nsplit = pl.nsplit; P.C = pl.C;
+  P.s_lo = pl.s_lo; P.n_hi = pl.n_hi;
   P.scale_log2 = p.scale * 1.4426950408889634f;
   P.cu_trunk = cu_trunk;
   P.anchors = anchors;
@@ -900,7 +968,7 @@ cudaError_t launch_attn_sm100(const AttnProblem& p, const void* q_br, const void
   cudaError_t e = cudaMemsetAsync(w + cnt_off, 0, pl.cnt_bytes, st);
   if (e != cudaSuccess) return e;
   const size_t smem = smem_bytes(p.D);
-  const dim3 grid((unsigned)((size_t)pl.ntile * p.Hkv * pl.nsplit));
+  const dim3 grid((unsigned)pl.units);
   if (p.D == 128) {
     e = cudaFuncSetAttribute(tree_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
