@@ -849,10 +849,11 @@ struct Plan {
 };
 
 // Work decomposition.  base = (query tile, kv head) pairs; each splits into
-// nsplit key chunks of C keys.  With fewer pairs than resident CTA slots
-// (SMs x 2), the smallest nsplit whose units fill every slot once: finer
-// chunks add per-unit prologue, epilogue and merge work.  With one to eight
-// waves of pairs, two chunks halve the tail of the last wave.
+// key chunks.  Branch pass with fewer pairs than resident CTA slots (SMs x
+// 2): one wave of units (the s_lo / n_hi split below, chunk sizes per pair
+// on the device).  Otherwise nsplit chunks of C keys: with one to eight
+// waves of pairs two chunks halve the tail of the last wave; the prefill
+// keeps one.
 Plan make_plan(const AttnProblem& p, int num_sms, bool prefill) {
   Plan pl;
   pl.RT = 128 / p.G;
